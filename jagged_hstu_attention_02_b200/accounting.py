@@ -1,0 +1,117 @@
+"""Host-side work accounting: valid pairs, FLOPs and algorithmic bytes.
+
+ - "Scaling HSTU: ragged execution, candidate amortization and content features",
+   section "Variable length is a central systems issue": padded vs ragged token
+   positions and the dense / per-sequence pair-work ratio (theoretical work only).
+ - The valid-pair count of one sequence follows the mask family named on
+   "HSTU-MUSA: HSTU for Moore Threads (MUSA)", section "Mathematical Equivalence",
+   in closed form (contextual prefix, causal history with an optional window W,
+   candidates that see the prefix, the history and themselves).
+
+FLOPs count valid (unmasked) pairs only:  fwd = P*H*2*(d_qk + d_v),
+bwd = P*H*2*(2*d_qk + 2*d_v) (no recompute); bwd_recompute = P*H*2*(3*d_qk + 2*d_v).
+"""
+from __future__ import annotations
+
+from fractions import Fraction
+
+import numpy as np
+
+
+def padding_stats(lengths):
+    """(padded token positions, ragged token positions, dense/per-sequence pair-work ratio)."""
+    lengths = [int(x) for x in lengths]
+    n = len(lengths)
+    m = max(lengths) if lengths else 0
+    padded = n * m
+    ragged = sum(lengths)
+    denom = sum(x * x for x in lengths)
+    ratio = Fraction(n * m * m, denom) if denom else Fraction(0)
+    return padded, ragged, ratio
+
+
+def _capped_triangle(n: int, K) -> int:
+    """sum_{m=1..n} min(m, K); K=None means no cap."""
+    if n <= 0:
+        return 0
+    if K is None or n <= K:
+        return n * (n + 1) // 2
+    return K * (K + 1) // 2 + (n - K) * K
+
+
+def valid_pairs_seq(L: int, c: int = 0, t: int = 0, W: int = 0) -> int:
+    """Number of valid (query, key) pairs of one sequence of length L."""
+    if L <= 0:
+        return 0
+    E = L - t
+    if E <= 0:
+        return L                       # only candidates: each sees itself
+    K = (W + 1) if W > 0 else None
+    hist = E - c
+    n = c * c                          # contextual rows see the contextual prefix
+    n += c * hist                      # history rows see every contextual key ...
+    n += _capped_triangle(hist, K)     # ... and causal (windowed) history keys
+    seen = hist if K is None else min(hist, K)
+    n += t * (1 + c + seen)            # candidates: themselves, the prefix, the last history keys
+    return n
+
+
+def valid_pairs(batch) -> int:
+    L = np.diff(batch.seq_offsets)
+    B = len(L)
+    c = batch.num_contextuals if batch.num_contextuals is not None else np.zeros(B, np.int32)
+    t = batch.num_targets if batch.num_targets is not None else np.zeros(B, np.int32)
+    return int(sum(valid_pairs_seq(int(L[b]), int(c[b]), int(t[b]), int(batch.max_attn_len))
+                   for b in range(B)))
+
+
+def fwd_flops(batch, pairs=None) -> int:
+    P = valid_pairs(batch) if pairs is None else pairs
+    return P * batch.num_heads * 2 * (batch.d_qk + batch.d_v)
+
+
+def bwd_flops(batch, pairs=None) -> int:
+    P = valid_pairs(batch) if pairs is None else pairs
+    return P * batch.num_heads * 2 * (2 * batch.d_qk + 2 * batch.d_v)
+
+
+def bwd_flops_recompute(batch, pairs=None) -> int:
+    P = valid_pairs(batch) if pairs is None else pairs
+    return P * batch.num_heads * 2 * (3 * batch.d_qk + 2 * batch.d_v)
+
+
+def elem_size(dtype: str) -> int:
+    return {"f32": 4, "bf16": 2}[dtype]
+
+
+def fwd_bytes(batch, training: bool = False) -> int:
+    """Algorithmic HBM bytes of one forward: read Q, K, V, U (+ timestamps, metadata,
+    tables), write O (+ fp32 Y, mean and rstd when training)."""
+    T, H, s = batch.total_tokens, batch.num_heads, elem_size(batch.dtype)
+    B = batch.batch
+    n = T * (2 * H * batch.d_qk + 2 * H * batch.d_v) * s   # Q, K, V, U
+    n += T * H * batch.d_v * s                               # O
+    if batch.time_bias_len > 0:
+        n += 8 * T
+    n += 8 * (B + 1) + 4 * B * 2
+    n += 4 * (batch.rel_bias_len + batch.time_bias_len)
+    if training:
+        n += 4 * T * H * batch.d_v + 8 * T
+    return n
+
+
+def bwd_bytes(batch) -> int:
+    """Algorithmic HBM bytes of one backward: read dO, Q, K, V, U, fp32 Y, mean, rstd
+    (+ timestamps, metadata, tables); write dQ, dK, dV, dU and the table gradients."""
+    T, H, s = batch.total_tokens, batch.num_heads, elem_size(batch.dtype)
+    B = batch.batch
+    D = H * batch.d_v
+    n = T * D * s                                            # dO
+    n += T * (2 * H * batch.d_qk + 2 * H * batch.d_v) * s    # Q, K, V, U
+    n += 4 * T * D + 8 * T                                   # Y, mean, rstd
+    n += T * (2 * H * batch.d_qk + 2 * H * batch.d_v) * s    # dQ, dK, dV, dU
+    if batch.time_bias_len > 0:
+        n += 8 * T
+    n += 8 * (B + 1) + 4 * B * 2
+    n += 2 * 4 * (batch.rel_bias_len + batch.time_bias_len)
+    return n
