@@ -1,0 +1,402 @@
+"""Benchmark of the jagged HSTU attention training step (forward + backward) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one pass of the whole path over one batch of the MovieLens-shaped training
+workload (B=128, H=4, d=128, bf16, Zipf history + 1 contextual + 1..20 candidate tokens,
+time and rel-pos bias, dO ~ N(0,1)): forward with saved activations, then backward.
+Throughput counts valid (unmasked) pairs only: fwd P*H*2*(d_qk+d_v) + bwd P*H*2*(2d_qk+2d_v).
+
+Prints ONE JSON line on rank 0.  Under torchrun each rank runs its own batch (seed + rank),
+no collective on the data path ("scaling": "weak"); timing is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from jagged_hstu_attention_02_b200 import accounting, synth  # noqa: E402
+
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+WORKLOAD_CFG = 4          # MovieLens-shaped inputs + upstream gradient
+SECONDARY_CFG = 2         # long-history forward (tensor-core regime)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms during the timed region."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", "hstu_clocks_%d_%d.csv" % (os.getpid(), gpu_index))
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.QUERY,
+                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        sm, smax, reasons = [], None, set()
+        names = ["active", "hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                 "sw_power_cap"]
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(names[1:], parts[5:9]):
+                if val.lower() in ("active", "1", "yes"):
+                    reasons.add(name)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def stage_timer(ops, torch, stages):
+    """Per-stage CUDA events recorded by the library around its kernels."""
+    evs = {}
+    for st in stages:
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        b.record()
+        ops.set_stage_events(st, a, b)
+        evs[st] = (a, b)
+    return evs
+
+
+def run_ours(args, world, rank, local):
+    import torch
+    from jagged_hstu_attention_02_b200 import ops
+
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    peaks, peak_kind = load_peaks()
+
+    b = synth.make_config(WORKLOAD_CFG, seed=synth.BASE_SEED + 1 + 1000 * rank)
+    P = accounting.valid_pairs(b)
+    flops = accounting.fwd_flops(b, P) + accounting.bwd_flops(b, P)
+    tokens = b.total_tokens
+    dev = ops.batch_to_device(b)
+    kw = ops.batch_kwargs(b)
+    out, saved = ops.run_fwd(b, dev, training=True)
+    grads = ops.run_bwd(b, saved, dev_tensors=dev)
+    ws_f = ops.fwd.last_workspace
+    ws_b = ops.bwd.last_workspace
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+
+    def step():
+        ops.fwd(dev["q"], dev["k"], dev["v"], dev["u"], dev["seq_offsets"],
+                dev["num_contextuals"], dev["num_targets"], dev["timestamps"], dev["rel_bias"],
+                dev["time_bias"], training=True, out=out, saved=saved, workspace=ws_f, **kw)
+        ops.bwd(dev["dout"], dev["q"], dev["k"], dev["v"], dev["u"], dev["seq_offsets"],
+                dev["num_contextuals"], dev["num_targets"], dev["timestamps"], dev["rel_bias"],
+                dev["time_bias"], saved=saved, grads=grads, workspace=ws_b, **kw)
+
+    stages = ["fwd_attn", "fwd_norm", "bwd_norm", "bwd_attn"]
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        step()
+    torch.cuda.synchronize()
+    evs = stage_timer(ops, torch, stages)
+    stage_ms = {s: [] for s in stages}
+    step_ms = []
+    clocks = ClockSampler(local)
+    clocks.start()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    t_region = time.perf_counter()
+    for _ in range(args.steps):
+        flush.fill_(1.0)                       # evict the previous step's data from L2
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        step()
+        e1.record()
+        e1.synchronize()
+        step_ms.append(e0.elapsed_time(e1))
+        for s in stages:
+            stage_ms[s].append(evs[s][0].elapsed_time(evs[s][1]))
+    torch.cuda.synchronize()
+    wall_region = time.perf_counter() - t_region
+    if world > 1:
+        torch.distributed.barrier()
+    clk = clocks.stop()
+    for s in stages:
+        ops.set_stage_events(s)
+    assert ops.read_device_status(ws_f) == 0 and ops.read_device_status(ws_b) == 0
+
+    ms = sum(step_ms) / len(step_ms)
+    if world > 1:
+        t = torch.tensor([ms], device="cuda")
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    value = world * flops / (ms * 1e-3) / 1e12
+
+    # roofline of the dominant kernel stage
+    avg = {s: sum(v) / len(v) for s, v in stage_ms.items()}
+    dom = max(avg, key=avg.get)
+    dom_bytes = {"fwd_attn": accounting.fwd_bytes(b, training=True),
+                 "fwd_norm": b.total_tokens * b.num_heads * b.d_v * (4 + 2 + 2) + 8 * tokens,
+                 "bwd_norm": b.total_tokens * b.num_heads * b.d_v * (2 + 2 + 4 + 2 + 4) + 8 * tokens,
+                 "bwd_attn": accounting.bwd_bytes(b)}[dom]
+    dom_flops = {"fwd_attn": accounting.fwd_flops(b, P), "bwd_attn": accounting.bwd_flops(b, P)}
+    hbm_peak = peaks["hbm_gbs"]
+    achieved = dom_bytes / (avg[dom] * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak,
+                "unit": "GB/s", "frac": round(achieved / hbm_peak, 4), "traffic": None,
+                "kernel_stage": dom, "kernel_ms": round(avg[dom], 4),
+                "peak_source": peak_kind, "stage_ms": {s: round(v, 4) for s, v in avg.items()}}
+    if dom in dom_flops:
+        roofline["tflops"] = round(dom_flops[dom] / (avg[dom] * 1e-3) / 1e12, 2)
+
+    # end to end through the public API with host buffers (pinned), copies inside the region
+    e2e = measure_e2e(args, b, ops, torch, kw, flops, world)
+
+    secondary = measure_secondary(ops, torch, peaks, rank) if rank == 0 and not args.quick else None
+    cpu = cpu_baseline(b) if (rank == 0 and world == 1 and not args.no_cpu) else None
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": "jagged HSTU attn fwd+bwd TFLOP/s (valid pairs) on 1 B200",
+        "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "tokens_per_s": round(world * tokens / (ms * 1e-3), 1),
+        "pct_bf16_peak": round(100 * value / world / peaks["bf16_tflops"], 3),
+        "config": {"workload": synth.WORKLOADS[WORKLOAD_CFG], "global_batch": b.batch * world,
+                   "tokens_per_gpu": tokens, "valid_pairs_per_gpu": P, "flops_per_step": flops,
+                   "max_seqlen": b.max_seqlen, "parallelism": "dp%d" % world,
+                   "l2": "flushed between steps (256 MB write), flush outside per-step events",
+                   "wall_s_region": round(wall_region, 3)},
+        "roofline": roofline, "e2e": e2e, "clocks": clk,
+        "gpu_launches": args.steps * LAUNCHES_PER_STEP,
+        "cpu_baseline": cpu, "secondary": secondary,
+    }
+    print(json.dumps(line), flush=True)
+
+
+# kernels of ours launched per step: fwd attention, fwd LayerNorm+gating, bwd LayerNorm+gating,
+# bwd attention, dQ conversion (memsets are not kernels of ours)
+LAUNCHES_PER_STEP = 5
+
+
+def measure_e2e(args, b, ops, torch, kw, flops, world):
+    host = {}
+    dt = torch.bfloat16 if b.dtype == "bf16" else torch.float32
+    src = dict(q=(b.q, dt), k=(b.k, dt), v=(b.v, dt), u=(b.u, dt), dout=(b.dout, dt),
+               seq_offsets=(b.seq_offsets, None), num_contextuals=(b.num_contextuals, None),
+               num_targets=(b.num_targets, None), timestamps=(b.timestamps, None),
+               rel_bias=(b.rel_bias, None), time_bias=(b.time_bias, None))
+    for name, (a, cast) in src.items():
+        t = torch.from_numpy(a)
+        if cast is not None:
+            t = t.to(cast)
+        host[name] = t.pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    dev = {n: torch.empty_like(t, device="cuda") for n, t in host.items()}
+    T, D = b.u.shape
+    out = torch.empty((T, D), dtype=dt, device="cuda")
+    saved = ops.Saved(torch.empty((T, D), device="cuda"), torch.empty(T, device="cuda"),
+                      torch.empty(T, device="cuda"))
+    grads = (torch.empty(b.q.shape, dtype=dt, device="cuda"),
+             torch.empty(b.k.shape, dtype=dt, device="cuda"),
+             torch.empty(b.v.shape, dtype=dt, device="cuda"),
+             torch.empty(b.u.shape, dtype=dt, device="cuda"),
+             torch.empty(b.rel_bias.shape, device="cuda"),
+             torch.empty(b.time_bias.shape, device="cuda"))
+    results = [out] + list(grads)
+    host_out = [torch.empty(r.shape, dtype=r.dtype, pin_memory=True) for r in results]
+    d2h = sum(t.numel() * t.element_size() for t in host_out)
+
+    def step():
+        for n in host:
+            dev[n].copy_(host[n], non_blocking=True)
+        ops.fwd(dev["q"], dev["k"], dev["v"], dev["u"], dev["seq_offsets"],
+                dev["num_contextuals"], dev["num_targets"], dev["timestamps"], dev["rel_bias"],
+                dev["time_bias"], training=True, out=out, saved=saved, **kw)
+        ops.bwd(dev["dout"], dev["q"], dev["k"], dev["v"], dev["u"], dev["seq_offsets"],
+                dev["num_contextuals"], dev["num_targets"], dev["timestamps"], dev["rel_bias"],
+                dev["time_bias"], saved=saved, grads=grads, **kw)
+        for r, h in zip(results, host_out):
+            h.copy_(r, non_blocking=True)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        step()
+    e1.record()
+    e1.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    return {"value": round(world * flops / (ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+            "ms_per_step": round(ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+def measure_secondary(ops, torch, peaks, rank):
+    """Long-history forward (the tensor-core regime): valid-pair TFLOP/s and % of bf16 peak."""
+    b = synth.make_config(SECONDARY_CFG)
+    P = accounting.valid_pairs(b)
+    fl = accounting.fwd_flops(b, P)
+    dev = ops.batch_to_device(b)
+    out = ops.run_fwd(b, dev)
+    ws = ops.fwd.last_workspace
+    kw = ops.batch_kwargs(b)
+    evs = stage_timer(ops, torch, ["fwd_attn"])
+    times, kt = [], []
+    for it in range(8):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        ops.fwd(dev["q"], dev["k"], dev["v"], dev["u"], dev["seq_offsets"],
+                dev["num_contextuals"], dev["num_targets"], dev["timestamps"], dev["rel_bias"],
+                dev["time_bias"], out=out, workspace=ws, **kw)
+        e1.record()
+        e1.synchronize()
+        if it >= 3:
+            times.append(e0.elapsed_time(e1))
+            kt.append(evs["fwd_attn"][0].elapsed_time(evs["fwd_attn"][1]))
+    ops.set_stage_events("fwd_attn")
+    ms = sum(times) / len(times)
+    kms = sum(kt) / len(kt)
+    tf = fl / (ms * 1e-3) / 1e12
+    ktf = fl / (kms * 1e-3) / 1e12
+    return {"workload": synth.WORKLOADS[SECONDARY_CFG], "metric": "fwd TFLOP/s (valid pairs)",
+            "value": round(tf, 2), "ms": round(ms, 4), "attn_kernel_ms": round(kms, 4),
+            "attn_kernel_tflops": round(ktf, 2),
+            "frac_of_bf16_peak": round(ktf / peaks["bf16_tflops"], 4),
+            "tokens_per_s": round(b.total_tokens / (ms * 1e-3), 1), "valid_pairs": P}
+
+
+def cpu_baseline(b, target_s=15.0):
+    """The fp64 oracle, as it stands, on a bounded sample of the workload's sequences."""
+    from oracle import oracle
+
+    order = list(range(b.batch))
+    n = max(1, b.batch // 8)
+    while True:
+        sb = synth.sub_batch(b, order[:n])
+        t0 = time.perf_counter()
+        oracle.fwd(sb)
+        oracle.bwd(sb)
+        el = time.perf_counter() - t0
+        if el > target_s / 4 or n >= b.batch:
+            break
+        n = min(b.batch, n * 2)
+    P = accounting.valid_pairs(sb)
+    fl = accounting.fwd_flops(sb, P) + accounting.bwd_flops(sb, P)
+    return {"value": round(fl / el / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
+            "kind": "oracle", "seconds": round(el, 3),
+            "sample": "first %d of %d sequences (%d tokens), fwd+bwd in fp64" %
+                      (n, b.batch, sb.total_tokens)}
+
+
+def run_reference(args, world, rank):
+    """The oracle timed on the host cores as the reference arm (rank 0 only)."""
+    if rank != 0:
+        return
+    from oracle import oracle
+
+    b = synth.make_config(WORKLOAD_CFG)
+    n = max(1, b.batch // 16)
+    sb = synth.sub_batch(b, list(range(n)))
+    P = accounting.valid_pairs(sb)
+    fl = accounting.fwd_flops(sb, P) + accounting.bwd_flops(sb, P)
+    for _ in range(min(args.warmup, 1)):
+        oracle.fwd(sb)
+        oracle.bwd(sb)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.fwd(sb)
+        oracle.bwd(sb)
+    el = (time.perf_counter() - t0) / args.steps
+    v = fl / el / 1e12
+    sample = "first %d of %d sequences per step (%d tokens), fwd+bwd in fp64" % (
+        n, b.batch, sb.total_tokens)
+    line = {"impl": "reference",
+            "metric": "jagged HSTU attn fwd+bwd TFLOP/s (valid pairs) on 1 B200",
+            "value": round(v, 6), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(el * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": synth.WORKLOADS[WORKLOAD_CFG], "global_batch": b.batch,
+                       "parallelism": "dp%d" % world},
+            "cpu_baseline": {"value": round(v, 6), "unit": "TFLOP/s",
+                             "cores": oracle.num_threads(), "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(v, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--quick", action="store_true", help="skip the long-history secondary line")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    world, rank, local = dist_setup(args)
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+    else:
+        run_ours(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,185 @@
+/*
+ * hstu_attn.h -- C ABI of the jagged HSTU attention library for NVIDIA B200 (sm_100a).
+ *
+ * The operation.  For every jagged sequence b (rows seq_offsets[b] .. seq_offsets[b+1]-1
+ * of the packed tensors, local positions 0..L-1), every head h and query row i:
+ *
+ *   s_ij = alpha * <q_i, k_j> + rel_bias[clamp(p(i) - p(j), 0, R-1)]
+ *                             + time_bias[min(floor(log(|ts[p(i)] - ts[p(j)]| + 1) / div), NB-1)]
+ *   A_ij = valid(i,j) ? SiLU(s_ij) / N : 0,            SiLU(x) = x * sigmoid(x)
+ *   Y_i  = sum_j A_ij V_j            (per head; heads concatenated into D = H * d_v features)
+ *   O_i  = U_i (.) LayerNorm(Y_i)    (over the D features, biased variance, eps, no affine)
+ *
+ * Sources (page title, section):
+ *  - "HSTU tensor by tensor: SiLU aggregation, temporal bias and gating", "Similar shape,
+ *    different aggregation": the pointwise SiLU aggregation A_ij = 1[j<=i] SiLU(q.k+b)/N
+ *    followed by U (.) Norm(sum_j A_ij V_j) (the W_o projection and residual that follow on
+ *    that page are not part of this library);
+ *  - same page, "SiLU aggregation coefficients are not probabilities" (SiLU = x*sigmoid(x)),
+ *    "Do not copy softmax masking mechanically" (illegal coefficients are zeroed after the
+ *    SiLU, never -inf before it), "Relative time adds information content similarity lacks"
+ *    and "Temporal bias is not simply fixed forgetting" (relative position and bucketed
+ *    elapsed-time bias), "Trace four projections" (d_qk may differ from d_v);
+ *  - "HSTU-MUSA: HSTU for Moore Threads (MUSA)", "Mathematical Equivalence": the mask family
+ *    (contextual bidirectional attention, candidate position clamping, target group
+ *    masking, max attention length); "Accuracy Alignment": N is the batch max_seqlen;
+ *  - "Scaling HSTU: ragged execution, candidate amortization and content features",
+ *    "Variable length is a central systems issue": jagged storage = values + offsets.
+ *
+ * The mask (c = num_contextuals[b], t = num_targets[b], E = L - t, W = max_attn_len):
+ *    p(x) = x for x < E, else E - 1 (candidates take the last history position; p(x) = x if E = 0)
+ *    valid(i,j) =  j >= E : i == j                      (candidate keys: seen by themselves only)
+ *                  i < c  : j < c                       (contextual rows: bidirectional prefix)
+ *                  j < c  : true                        (contextual keys: seen by every row)
+ *                  else   : j <= p(i) && (W <= 0 || p(i) - j <= W)
+ *
+ * Layouts (all row-major, packed over the T = seq_offsets[B] tokens of the batch):
+ *    q, k        [T, H, d_qk]        dtype            dq, dk   [T, H, d_qk]  dtype
+ *    v           [T, H, d_v]         dtype            dv       [T, H, d_v]   dtype
+ *    u, out      [T, H * d_v]        dtype            du, dout [T, H * d_v]  dtype
+ *    saved_y     [T, H * d_v]        fp32 (Y, already scaled by 1/N)
+ *    saved_mean, saved_rstd [T]      fp32
+ *    seq_offsets [B + 1] int64 (seq_offsets[0] = 0, non-decreasing, seq_offsets[B] = T)
+ *    num_contextuals, num_targets [B] int32 (NULL = all zero)
+ *    timestamps  [T] int64, in the caller's integer time unit (NULL allowed when NB = 0);
+ *                |ts_i - ts_j| within a sequence must be below 2^63
+ *    rel_bias [R], time_bias [NB], d_rel_bias [R], d_time_bias [NB]  fp32
+ *
+ * Ownership and synchronisation.  The caller allocates every buffer, including the
+ * workspace.  fwd/bwd allocate nothing, never synchronise, and only enqueue work on
+ * `stream` (a cudaStream_t; NULL = the legacy default stream).  All array pointers are
+ * device pointers; `params` is a host pointer read before the call returns.  Device
+ * pointers must be 16-byte aligned.
+ *
+ * Errors.  Host-checkable problems (NULL required pointer, sizes out of range, misaligned
+ * pointer, workspace too small) return a status before anything is enqueued.  Problems in
+ * device-resident data (offsets not monotone or not ending at T, c + t > L, L > max_seqlen)
+ * are not fatal: the offending sequence is skipped and a bit is set in the status word at
+ * the start of the workspace; hstu_attn_read_device_status() reads it.  No kernel traps,
+ * and every wait inside a kernel is bounded.
+ */
+#ifndef HSTU_ATTN_H
+#define HSTU_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    HSTU_OK = 0,
+    HSTU_ERR_INVALID_ARGUMENT = 1,   /* bad pointer, size, alignment or parameter */
+    HSTU_ERR_UNSUPPORTED = 2,        /* valid request outside the compiled kernel set */
+    HSTU_ERR_WORKSPACE_TOO_SMALL = 3,
+    HSTU_ERR_CUDA = 4,               /* a CUDA runtime call or launch failed */
+    HSTU_ERR_DEVICE_DATA = 5         /* returned by hstu_attn_read_device_status only */
+} hstu_status_t;
+
+typedef enum { HSTU_F32 = 0, HSTU_BF16 = 1 } hstu_dtype_t;
+
+/* Bits of the device status word. */
+#define HSTU_DEV_BAD_OFFSETS   0x1   /* seq_offsets not non-decreasing / not ending at T */
+#define HSTU_DEV_BAD_COUNTS    0x2   /* num_contextuals/num_targets negative or c + t > L */
+#define HSTU_DEV_SEQ_TOO_LONG  0x4   /* a sequence longer than max_seqlen */
+#define HSTU_DEV_WAIT_TIMEOUT  0x8   /* a bounded in-kernel wait gave up */
+
+typedef struct {
+    int32_t batch;            /* B >= 0 */
+    int32_t num_heads;        /* H >= 1 */
+    int32_t d_qk;             /* 1..256 (f32); multiple of 16 in 16..128 (bf16) */
+    int32_t d_v;              /* as d_qk; H * d_v <= 2048 */
+    int32_t max_seqlen;       /* N >= 1: the batch max of L; the 1/N scale. Host never reads offsets */
+    int32_t max_attn_len;     /* W; <= 0 means unlimited */
+    int64_t total_tokens;     /* T = seq_offsets[B] */
+    float alpha;              /* score scale on q.k (not on the bias) */
+    float ln_eps;             /* LayerNorm epsilon, e.g. 1e-5 */
+    int32_t rel_bias_len;     /* R >= 0; 0 = no relative-position bias */
+    int32_t time_bias_len;    /* NB in 0..256; 0 = no time bias (timestamps may be NULL) */
+    double time_bucket_div;   /* > 0, e.g. 0.301 (natural log) */
+    int32_t dtype;            /* hstu_dtype_t of q,k,v,u,out,dout,dq,dk,dv,du */
+    int32_t reserved;         /* must be 0 */
+} hstu_attn_params_t;
+
+/* Workspace bytes hstu_attn_fwd needs for these params (saved_y NULL or not). */
+hstu_status_t hstu_attn_fwd_workspace_size(const hstu_attn_params_t *params, size_t *bytes);
+
+/*
+ * Forward.  Writes out; when saved_y is non-NULL also writes saved_y, saved_mean and
+ * saved_rstd (all three or none), which hstu_attn_bwd consumes.
+ */
+hstu_status_t hstu_attn_fwd(const hstu_attn_params_t *params, const void *q, const void *k,
+                            const void *v, const void *u, const int64_t *seq_offsets,
+                            const int32_t *num_contextuals, const int32_t *num_targets,
+                            const int64_t *timestamps, const float *rel_bias,
+                            const float *time_bias, void *out, float *saved_y,
+                            float *saved_mean, float *saved_rstd, void *workspace,
+                            size_t workspace_bytes, void *stream);
+
+/* Workspace bytes hstu_attn_bwd needs for these params. */
+hstu_status_t hstu_attn_bwd_workspace_size(const hstu_attn_params_t *params, size_t *bytes);
+
+/*
+ * Backward of loss = sum(dout (.) out).  Inputs as for the forward plus dout and the
+ * saved_y/mean/rstd written by the forward on the same inputs.  Overwrites dq, dk, dv, du
+ * and (when the table is present) d_rel_bias / d_time_bias.
+ */
+hstu_status_t hstu_attn_bwd(const hstu_attn_params_t *params, const void *dout, const void *q,
+                            const void *k, const void *v, const void *u,
+                            const int64_t *seq_offsets, const int32_t *num_contextuals,
+                            const int32_t *num_targets, const int64_t *timestamps,
+                            const float *rel_bias, const float *time_bias, const float *saved_y,
+                            const float *saved_mean, const float *saved_rstd, void *dq, void *dk,
+                            void *dv, void *du, float *d_rel_bias, float *d_time_bias,
+                            void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Reads the device status word at the start of `workspace` after the work queued on
+ * `stream` finishes (synchronises `stream`).  *code receives the HSTU_DEV_* bits (0 = ok).
+ * Returns HSTU_ERR_DEVICE_DATA when *code != 0.
+ */
+hstu_status_t hstu_attn_read_device_status(const void *workspace, void *stream, int32_t *code);
+
+/*
+ * Test hook: writes the mask of sequence `seq` as evaluated by the device predicate the
+ * kernels use, row-major bits (bit j of row i at word (i*L + j) / 32, bit (i*L + j) % 32),
+ * into `bits` (device, ceil(L*L/32) words, L = seq_offsets[seq+1]-seq_offsets[seq] which the
+ * caller passes as seq_len).  Enqueued on `stream`.
+ */
+hstu_status_t hstu_attn_debug_mask(const hstu_attn_params_t *params, const int64_t *seq_offsets,
+                                   const int32_t *num_contextuals, const int32_t *num_targets,
+                                   int32_t seq, int32_t seq_len, uint32_t *bits, void *stream);
+
+/*
+ * Host helper: the time-bucket thresholds the device compares against.  out[k-1] is the
+ * smallest |dt| whose bucket is >= k, for k = 1..nb-1, with the bucket decided in fp64
+ * exactly as floor(log((double)|dt| + 1.0) / div) (UINT64_MAX when never reached).
+ */
+hstu_status_t hstu_attn_time_thresholds(double div, int32_t nb, uint64_t *out);
+
+/* Kernel stages of fwd/bwd, for hstu_attn_set_stage_events. */
+#define HSTU_STAGE_FWD_ATTN 0   /* forward attention (scores, bias, SiLU, mask, A V) */
+#define HSTU_STAGE_FWD_NORM 1   /* forward LayerNorm + U gating */
+#define HSTU_STAGE_BWD_NORM 2   /* backward of LayerNorm + U gating (dU, dY) */
+#define HSTU_STAGE_BWD_ATTN 3   /* backward attention (dQ, dK, dV, table gradients) */
+#define HSTU_NUM_STAGES 4
+
+/*
+ * Measurement hook.  While set, every fwd/bwd call records `start_event` on its stream just
+ * before launching the kernel(s) of `stage` and `stop_event` just after (both cudaEvent_t).
+ * NULL events clear the hook.  Process-wide and not thread-safe: for benchmarks only.
+ */
+hstu_status_t hstu_attn_set_stage_events(int32_t stage, void *start_event, void *stop_event);
+
+/* Static description of a status code. */
+const char *hstu_status_string(hstu_status_t status);
+
+/* Library version, e.g. 100 for 0.1.0. */
+int32_t hstu_attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HSTU_ATTN_H */

@@ -1,0 +1,158 @@
+// common.cuh -- device-side definitions shared by the jagged HSTU attention kernels.
+//
+// The mask family and bias follow "HSTU-MUSA: HSTU for Moore Threads (MUSA)",
+// section "Mathematical Equivalence" (contextual bidirectional prefix, candidate position
+// clamping, target group masking, max attention length) and "HSTU tensor by tensor: SiLU
+// aggregation, temporal bias and gating", sections "Relative time adds information content
+// similarity lacks" and "Do not copy softmax masking mechanically".  The exact reading of
+// each rule is stated in include/hstu_attn.h.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/hstu_attn.h"
+
+namespace hstu {
+
+constexpr int kMaxTimeBuckets = 256;
+
+// Everything a kernel needs, passed by value as a __grid_constant__ parameter.
+struct DevParams {
+    int32_t B, H, dqk, dv, N, W;
+    int64_t T;
+    int32_t D;            // H * dv
+    float alpha, inv_N, eps;
+    int32_t R, NB;
+    int32_t n_thr;        // reachable thresholds (<= NB - 1)
+    const int64_t *offsets;
+    const int32_t *ctx, *tgt;
+    const int64_t *ts;
+    const float *rel, *tb;
+    int32_t *status;
+    // smallest |dt| of bucket k+1 (fp64-decided on the host), ascending
+    uint64_t thr[kMaxTimeBuckets - 1];
+};
+
+struct SeqInfo {
+    int64_t start;
+    int L, c, t, E;
+    bool ok;
+};
+
+__device__ __forceinline__ void flag_error(const DevParams &p, int bits)
+{
+    atomicOr(p.status, bits);
+}
+
+// Reads and validates sequence b.  Invalid sequences are reported and skipped.
+__device__ __forceinline__ SeqInfo load_seq(const DevParams &p, int b, bool report)
+{
+    SeqInfo s;
+    int64_t a = p.offsets[b], e = p.offsets[b + 1];
+    int64_t L = e - a;
+    s.start = a;
+    s.c = p.ctx ? p.ctx[b] : 0;
+    s.t = p.tgt ? p.tgt[b] : 0;
+    s.ok = true;
+    int bits = 0;
+    if (a < 0 || L < 0 || e > p.T) { bits |= HSTU_DEV_BAD_OFFSETS; }
+    if (L > p.N) { bits |= HSTU_DEV_SEQ_TOO_LONG; }
+    if (bits == 0 && (s.c < 0 || s.t < 0 || (int64_t)s.c + s.t > L)) bits |= HSTU_DEV_BAD_COUNTS;
+    if (bits) {
+        s.ok = false;
+        if (report) flag_error(p, bits);
+        L = 0;
+    }
+    s.L = (int)L;
+    s.E = s.L - s.t;
+    return s;
+}
+
+// p(x): candidates take the last history position.
+__device__ __forceinline__ int clamp_pos(int x, int E) { return (E > 0 && x >= E) ? E - 1 : x; }
+
+__device__ __forceinline__ bool pair_valid(int i, int j, const SeqInfo &s, int W)
+{
+    if (j >= s.E) return i == j;          // candidate key: itself only
+    if (i < s.c) return j < s.c;          // contextual row: bidirectional prefix
+    if (j < s.c) return true;             // contextual key: every row
+    int pi = clamp_pos(i, s.E);
+    return j <= pi && (W <= 0 || pi - j <= W);
+}
+
+// True when some pair of rows [i0,i1] x keys [j0,j1] (inclusive) is valid.  Never false
+// for a tile that holds a valid pair.
+__device__ __forceinline__ bool tile_any_valid(int i0, int i1, int j0, int j1, const SeqInfo &s,
+                                               int W)
+{
+    i1 = min(i1, s.L - 1);
+    j1 = min(j1, s.L - 1);
+    if (i0 > i1 || j0 > j1) return false;
+    if (j0 < s.c) return true;                              // contextual keys: every row
+    int a = max(j0, s.E);
+    if (a <= j1 && max(i0, a) <= min(i1, j1)) return true;  // candidate diagonal
+    int ha = max(j0, s.c), hb = min(j1, s.E - 1);           // history keys
+    if (ha > hb) return false;
+    int ra = max(i0, s.c), rb = min(i1, s.E - 1);           // history rows
+    if (ra <= rb && rb >= ha && (W <= 0 || ra - hb <= W)) return true;
+    if (i1 >= s.E && (W <= 0 || (s.E - 1) - hb <= W)) return true;   // candidate rows
+    return false;
+}
+
+// True when every pair of the (in-sequence) tile is valid and no pair needs the
+// candidate clamp: the bias then is rel[i-j] + tb[bucket(|ts_i - ts_j|)] without clamping
+// of positions.  Conservative: may return false for a full tile.
+__device__ __forceinline__ bool tile_all_valid(int i0, int i1, int j0, int j1, const SeqInfo &s,
+                                               int W)
+{
+    if (i1 >= s.L || j1 >= s.L || i1 >= s.E) return false;
+    if (j1 < s.c) return true;                               // all contextual keys
+    if (i0 < s.c || j1 >= s.E) return false;
+    // history x history (or contextual keys): needs j <= i for all, window for all
+    int jmin_hist = max(j0, s.c);
+    if (j1 > i0) return false;
+    if (W > 0 && i1 - jmin_hist > W) return false;
+    return true;
+}
+
+__device__ __forceinline__ uint64_t abs_diff_u64(int64_t a, int64_t b)
+{
+    return a >= b ? (uint64_t)a - (uint64_t)b : (uint64_t)b - (uint64_t)a;
+}
+
+// Number of thresholds <= dt (thresholds ascending, in shared or constant memory).
+__device__ __forceinline__ int bucket_search(const uint64_t *thr, int n, uint64_t dt)
+{
+    int lo = 0, hi = n;
+    while (lo < hi) {
+        int mid = (lo + hi) >> 1;
+        if (thr[mid] <= dt) lo = mid + 1; else hi = mid;
+    }
+    return lo;
+}
+
+template <typename T> __device__ __forceinline__ float to_f32(T x);
+template <> __device__ __forceinline__ float to_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x)
+{
+    return __bfloat162float(x);
+}
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x)
+{
+    return __float2bfloat16_rn(x);
+}
+
+__device__ __forceinline__ float silu_f32(float x) { return x / (1.0f + expf(-x)); }
+
+__device__ __forceinline__ float silu_grad_f32(float x)
+{
+    float sg = 1.0f / (1.0f + expf(-x));
+    return sg * (1.0f + x * (1.0f - sg));
+}
+
+}  // namespace hstu

@@ -190,6 +190,28 @@ def make_config(cfg: int, seed: Optional[int] = None) -> Batch:
     raise ValueError("unknown workload %r" % cfg)
 
 
+def sub_batch(b, seqs):
+    """The sequences `seqs` of batch b as a batch of their own (same N, same tables)."""
+    seqs = list(seqs)
+    offs = b.seq_offsets
+    rows = np.concatenate([np.arange(offs[s], offs[s + 1]) for s in seqs]) if seqs else \
+        np.zeros(0, dtype=np.int64)
+    lengths = np.array([offs[s + 1] - offs[s] for s in seqs], dtype=np.int64)
+    new_offs = np.zeros(len(seqs) + 1, dtype=np.int64)
+    new_offs[1:] = np.cumsum(lengths)
+
+    def pick(a):
+        return None if a is None else np.ascontiguousarray(a[rows])
+
+    def pick_seq(a):
+        return None if a is None else np.ascontiguousarray(a[seqs])
+
+    return dataclasses.replace(
+        b, seq_offsets=new_offs, num_contextuals=pick_seq(b.num_contextuals),
+        num_targets=pick_seq(b.num_targets), timestamps=pick(b.timestamps), q=pick(b.q),
+        k=pick(b.k), v=pick(b.v), u=pick(b.u), dout=pick(b.dout))
+
+
 def draw_dout(batch: Batch, seed: int) -> np.ndarray:
     """An upstream gradient dO ~ N(0,1) in the batch dtype, from its own seed."""
     rng = np.random.default_rng(seed)

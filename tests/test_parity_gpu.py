@@ -1,0 +1,258 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle, element by element.
+
+Tolerances: max|err| <= 1e-2*max|ref| + 1e-3 for bf16 inputs, <= 1e-5*max|ref| for fp32
+inputs, per output tensor; the masked-pair structure bit-exact.
+"""
+import numpy as np
+import pytest
+import torch
+
+from jagged_hstu_attention_02_b200 import ops, synth
+from oracle import oracle
+from tests.helpers import assert_close, rows_of, sub_batch
+
+pytestmark = pytest.mark.gpu
+
+
+def _np(t):
+    return t.detach().float().cpu().numpy()
+
+
+def _fwd_check(b, training=True, what=""):
+    dev = ops.batch_to_device(b)
+    if training:
+        out, saved = ops.run_fwd(b, dev, training=True)
+    else:
+        out = ops.run_fwd(b, dev)
+    torch.cuda.synchronize()
+    ref = oracle.fwd(b)
+    assert_close(_np(out), ref["out"], b.dtype, what + " out")
+    if training:
+        assert_close(_np(saved.y), ref["y"], b.dtype, what + " y")
+        assert_close(_np(saved.mean), ref["mean"], b.dtype, what + " mean")
+        # rstd is large where Y is tiny; compare it relative to itself
+        assert_close(_np(saved.rstd), ref["rstd"], b.dtype, what + " rstd")
+    assert ops.read_device_status(ops.fwd.last_workspace) == 0
+    return dev, out
+
+
+SMALL_CASES = [
+    # name, lengths, H, dqk, dv, dtype, ctx, tgt, W, R, NB
+    ("f32-causal", [1, 37, 129, 300, 0, 513], 2, 32, 32, "f32", 0, 0, 0, 514, 0),
+    ("f32-full-family", [5, 200, 77, 260], 2, 48, 80, "f32", [1, 4, 0, 8], [2, 20, 5, 0], 0,
+     261, 128),
+    ("f32-window", [300, 130, 2], 1, 32, 32, "f32", [3, 3, 1], [7, 0, 1], 17, 40, 64),
+    ("bf16-causal", [1, 37, 129, 300, 0, 513], 2, 64, 64, "bf16", 0, 0, 0, 514, 128),
+    ("bf16-family", [5, 200, 77, 260, 129], 4, 128, 128, "bf16", [1, 4, 0, 8, 3],
+     [2, 20, 5, 0, 64], 0, 261, 128),
+    ("bf16-window", [700, 130, 2, 256], 2, 64, 64, "bf16", [8, 8, 1, 8], [32, 0, 1, 248], 100,
+     101, 128),
+    ("bf16-small-window", [400], 2, 32, 32, "bf16", 2, 10, 5, 8, 128),
+    ("bf16-all-targets", [64, 150], 2, 64, 64, "bf16", 0, [64, 150], 0, 10, 128),
+    ("bf16-all-context", [64, 150], 2, 64, 64, "bf16", [64, 150], 0, 0, 151, 128),
+    ("bf16-dqk-ne-dv", [90, 300], 2, 128, 64, "bf16", 1, 3, 0, 301, 128),
+]
+
+
+@pytest.mark.parametrize("case", SMALL_CASES, ids=[c[0] for c in SMALL_CASES])
+def test_fwd_parity_small(case):
+    name, lengths, H, dqk, dv, dtype, ctx, tgt, W, R, NB = case
+    b = synth.make_batch(np.random.default_rng(100), lengths, H, dqk, dv, dtype,
+                         contextuals=ctx, targets=tgt, max_attn_len=W, rel_bias_len=R,
+                         time_bias_len=NB)
+    _fwd_check(b, what=name)
+
+
+@pytest.mark.parametrize("case", SMALL_CASES, ids=[c[0] for c in SMALL_CASES])
+def test_bwd_parity_small(case):
+    name, lengths, H, dqk, dv, dtype, ctx, tgt, W, R, NB = case
+    b = synth.make_batch(np.random.default_rng(101), lengths, H, dqk, dv, dtype,
+                         contextuals=ctx, targets=tgt, max_attn_len=W, rel_bias_len=R,
+                         time_bias_len=NB, with_dout=True)
+    dev = ops.batch_to_device(b)
+    out, saved = ops.run_fwd(b, dev, training=True)
+    dq, dk, dv_, du, drel, dtb = ops.run_bwd(b, saved, dev_tensors=dev)
+    torch.cuda.synchronize()
+    assert ops.read_device_status(ops.bwd.last_workspace) == 0
+    ref = oracle.bwd(b)
+    assert_close(_np(dq), ref["dq"], dtype, name + " dq")
+    assert_close(_np(dk), ref["dk"], dtype, name + " dk")
+    assert_close(_np(dv_), ref["dv"], dtype, name + " dv")
+    assert_close(_np(du), ref["du"], dtype, name + " du")
+    if R > 0:
+        assert_close(_np(drel), ref["drel"], dtype, name + " drel")
+    if NB > 0:
+        assert_close(_np(dtb), ref["dtb"], dtype, name + " dtb")
+
+
+# ------------------------------------------------------------------ the five workloads
+
+def test_fwd_parity_tiny_fp32_workload():
+    _fwd_check(synth.make_config(0), what="tiny fp32")
+
+
+def test_fwd_parity_movielens_workload():
+    _fwd_check(synth.make_config(1), what="movielens-shaped")
+
+
+@pytest.mark.parametrize("cfg", [2, 3])
+def test_fwd_parity_long_workloads_sampled(cfg):
+    """Full-size batch on the GPU; the oracle checks whole sequences sampled from it
+    (shortest, longest and one in between), which are independent given N."""
+    b = synth.make_config(cfg)
+    dev = ops.batch_to_device(b)
+    out = ops.run_fwd(b, dev)
+    torch.cuda.synchronize()
+    assert ops.read_device_status(ops.fwd.last_workspace) == 0
+    L = b.lengths
+    seqs = sorted({int(np.argmin(L)), int(np.argmax(L)), int(np.argsort(L)[len(L) // 2])})
+    ref = oracle.fwd(sub_batch(b, seqs))
+    got = _np(out)[rows_of(b, seqs)]
+    assert_close(got, ref["out"], b.dtype, "workload %d sampled out" % cfg)
+
+
+def test_bwd_parity_tiny_fp32_workload():
+    b = synth.make_config(0)
+    b.dout = synth.draw_dout(b, 777)
+    dev = ops.batch_to_device(b)
+    _, saved = ops.run_fwd(b, dev, training=True)
+    g = ops.run_bwd(b, saved, dev_tensors=dev)
+    ref = oracle.bwd(b)
+    for got, key in zip(g, ["dq", "dk", "dv", "du", "drel"]):
+        assert_close(_np(got), ref[key], "f32", "tiny fp32 " + key)
+
+
+def test_bwd_parity_training_workload():
+    b = synth.make_config(4)
+    dev = ops.batch_to_device(b)
+    _, saved = ops.run_fwd(b, dev, training=True)
+    g = ops.run_bwd(b, saved, dev_tensors=dev)
+    torch.cuda.synchronize()
+    assert ops.read_device_status(ops.bwd.last_workspace) == 0
+    ref = oracle.bwd(b)
+    for got, key in zip(g, ["dq", "dk", "dv", "du", "drel", "dtb"]):
+        assert_close(_np(got), ref[key], "bf16", "training workload " + key)
+
+
+# ------------------------------------------------------------------ mask structure
+
+MASK_CASES = [(1, 0, 0, 0), (5, 2, 3, 0), (130, 4, 64, 0), (300, 8, 32, 50), (257, 0, 0, 0),
+              (64, 64, 0, 0), (20, 0, 20, 0), (129, 1, 20, 1), (400, 3, 5, 127), (0, 0, 0, 0)]
+
+
+@pytest.mark.parametrize("W", [0, 50])
+def test_debug_mask_bit_exact(W):
+    lengths = [c[0] for c in MASK_CASES]
+    ctx = np.array([c[1] for c in MASK_CASES], np.int32)
+    tgt = np.array([c[2] for c in MASK_CASES], np.int32)
+    offs = np.zeros(len(lengths) + 1, np.int64)
+    offs[1:] = np.cumsum(lengths)
+    d_offs = torch.from_numpy(offs).cuda()
+    d_ctx = torch.from_numpy(ctx).cuda()
+    d_tgt = torch.from_numpy(tgt).cuda()
+    p = ops.Params(batch=len(lengths), num_heads=1, d_qk=16, d_v=16, max_seqlen=max(lengths),
+                   max_attn_len=W, total_tokens=int(offs[-1]), alpha=1.0, ln_eps=1e-5,
+                   rel_bias_len=0, time_bias_len=0, time_bucket_div=0.301, dtype=ops.HSTU_BF16,
+                   reserved=0)
+    for s, L in enumerate(lengths):
+        got = ops.debug_mask(p, d_offs, d_ctx, d_tgt, s, L).numpy()
+        ref, _ = oracle.mask(L, int(ctx[s]), int(tgt[s]), W)
+        assert np.array_equal(got, ref.astype(bool)), (s, L, W)
+
+
+# ------------------------------------------------------------------ page example on the GPU
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_page_signed_aggregation_on_gpu(dtype):
+    """q_1 = e0, k_0 = -e0, k_1 = e0, V_0 = e0, V_1 = e1, zero biases: N*Y_1 = [SiLU(-1), SiLU(1)]
+    ~ [-0.269, 0.731] as printed on the HSTU tensor-by-tensor page."""
+    b = synth.make_batch(np.random.default_rng(0), [2], 1, 32, 32, dtype, rel_bias_len=0,
+                         alpha=1.0)
+    for a in (b.q, b.k, b.v):
+        a[...] = 0.0
+    b.u[...] = 1.0
+    b.q[1, 0, 0] = 1.0
+    b.k[0, 0, 0] = -1.0
+    b.k[1, 0, 0] = 1.0
+    b.v[0, 0, 0] = 1.0
+    b.v[1, 0, 1] = 1.0
+    _, saved = ops.run_fwd(b, training=True)
+    y = _np(saved.y) * b.max_seqlen
+    tol = 1e-5 if dtype == "f32" else 4e-3
+    assert abs(y[1, 0] - (-0.269)) < 5e-4 + tol and abs(y[1, 1] - 0.731) < 5e-4 + tol
+    assert np.all(y[0] == 0.0)
+
+
+# ------------------------------------------------------------------ invariants
+
+def test_changing_future_inputs_leaves_earlier_outputs_bitwise_unchanged():
+    b = synth.make_batch(np.random.default_rng(5), [700, 300], 2, 64, 64, "bf16", contextuals=4,
+                         targets=[16, 8], rel_bias_len=701, time_bias_len=128)
+    out0 = _np(ops.run_fwd(b))
+    for cut in [130, 400]:
+        b2 = synth.make_batch(np.random.default_rng(5), [700, 300], 2, 64, 64, "bf16",
+                              contextuals=4, targets=[16, 8], rel_bias_len=701, time_bias_len=128)
+        rng = np.random.default_rng(cut)
+        for name in ("q", "k", "v", "u"):
+            a = getattr(b2, name)
+            a[cut + 1:700] = synth.round_to_dtype(
+                rng.standard_normal(a[cut + 1:700].shape).astype(np.float32), "bf16")
+        b2.timestamps[cut + 1:700] += 1000
+        out1 = _np(ops.run_fwd(b2))
+        assert np.array_equal(out0[:cut + 1], out1[:cut + 1]), cut
+        assert np.array_equal(out0[700:], out1[700:])        # other sequence untouched
+
+
+def test_candidate_isolation_bitwise():
+    b = synth.make_batch(np.random.default_rng(6), [300], 2, 64, 64, "bf16", contextuals=2,
+                         targets=20, rel_bias_len=301, time_bias_len=128)
+    out0 = _np(ops.run_fwd(b))
+    m = 290
+    for name in ("q", "k", "v", "u"):
+        getattr(b, name)[m] *= -1.0
+    out1 = _np(ops.run_fwd(b))
+    others = [i for i in range(300) if i != m]
+    assert np.array_equal(out0[others], out1[others])
+
+
+def test_forward_is_deterministic():
+    b = synth.make_config(1)
+    dev = ops.batch_to_device(b)
+    a = ops.run_fwd(b, dev).clone()
+    c = ops.run_fwd(b, dev)
+    assert torch.equal(a, c)
+
+
+# ------------------------------------------------------------------ edge cases and faults
+
+def test_empty_batch_and_zero_length_sequences():
+    b = synth.make_batch(np.random.default_rng(8), [0, 0, 3, 0], 2, 64, 64, "bf16",
+                         rel_bias_len=4, time_bias_len=128)
+    _fwd_check(b, what="zero-length")
+    dev = ops.batch_to_device(b)
+    e = synth.make_batch(np.random.default_rng(8), [], 2, 64, 64, "bf16", rel_bias_len=4,
+                         max_seqlen=1)
+    out = ops.run_fwd(e)
+    assert out.shape == (0, 128)
+    del dev
+
+
+def test_bad_device_data_is_reported_and_the_context_stays_usable():
+    b = synth.make_batch(np.random.default_rng(9), [10, 20, 30], 2, 64, 64, "bf16",
+                         contextuals=[1, 2, 3], targets=[1, 2, 3], rel_bias_len=31,
+                         time_bias_len=128)
+    dev = ops.batch_to_device(b)
+    bad = dict(dev)
+    bad["num_targets"] = torch.tensor([1, 25, 3], dtype=torch.int32, device="cuda")   # c+t > L
+    ops.run_fwd(b, bad)
+    assert ops.read_device_status(ops.fwd.last_workspace) & ops.DEV_BAD_COUNTS
+    bad = dict(dev)
+    bad["seq_offsets"] = torch.tensor([0, 10, 5, 60], dtype=torch.int64, device="cuda")
+    ops.run_fwd(b, bad)
+    assert ops.read_device_status(ops.fwd.last_workspace) & ops.DEV_BAD_OFFSETS
+    short = dict(alpha=b.alpha, max_seqlen=20, max_attn_len=0)
+    ops.fwd(dev["q"], dev["k"], dev["v"], dev["u"], dev["seq_offsets"], dev["num_contextuals"],
+            dev["num_targets"], dev["timestamps"], dev["rel_bias"], dev["time_bias"], **short)
+    assert ops.read_device_status(ops.fwd.last_workspace) & ops.DEV_SEQ_TOO_LONG
+    # a valid call afterwards still matches the oracle
+    _fwd_check(b, what="after bad data")
