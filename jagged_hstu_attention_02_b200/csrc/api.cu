@@ -242,8 +242,12 @@ hstu_status_t hstu_attn_fwd(const hstu_attn_params_t *p, const void *q, const vo
                      : reinterpret_cast<float *>(reinterpret_cast<char *>(workspace) + kHeaderBytes);
     {
         StageScope scope(HSTU_STAGE_FWD_ATTN, s);
-        if (p->dtype == HSTU_F32) HSTU_CUDA_TRY(launch_simt_fwd<float>(d, q, k, v, y, s));
-        else HSTU_CUDA_TRY(launch_simt_fwd<__nv_bfloat16>(d, q, k, v, y, s));
+        if (p->dtype == HSTU_F32)
+            HSTU_CUDA_TRY(launch_simt_fwd<float>(d, q, k, v, y, s));
+        else if (tc_fwd_supported(p->d_qk, p->d_v, p->total_tokens))
+            HSTU_CUDA_TRY(launch_tc_fwd(d, q, k, v, y, s));
+        else
+            HSTU_CUDA_TRY(launch_simt_fwd<__nv_bfloat16>(d, q, k, v, y, s));
     }
     {
         StageScope scope(HSTU_STAGE_FWD_NORM, s);

@@ -25,6 +25,11 @@ cudaError_t launch_simt_bwd(const DevParams &p, const void *q, const void *k, co
 template <typename T>
 cudaError_t launch_convert(const float *src, void *dst, int64_t n, cudaStream_t st);
 
+// tcgen05 forward attention (bf16): Y = (1/N) sum_j A_ij V_j in fp32.
+bool tc_fwd_supported(int dqk, int dv, int64_t T);
+cudaError_t launch_tc_fwd(const DevParams &p, const void *q, const void *k, const void *v,
+                          float *y, cudaStream_t st);
+
 cudaError_t launch_debug_mask(const DevParams &p, int seq, int seq_len, uint32_t *bits,
                               cudaStream_t st);
 
