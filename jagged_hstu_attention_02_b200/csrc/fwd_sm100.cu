@@ -1,21 +1,29 @@
 // fwd_sm100.cu -- tensor-core (tcgen05) forward attention of jagged HSTU for B200.
 //
-// One CTA per (128-row query tile, sequence, head).  Per key tile of 128 that holds a valid
-// pair:  S = Q K^T on tcgen05 (bf16 operands staged by TMA in 128-byte-swizzled shared
-// memory, fp32 accumulator in TMEM), then the epilogue warps read S from TMEM and form
-// A = mask ? SiLU(alpha*S + b) : 0 in fp32 (bias = relative-position + bucketed time table
-// entries; the mask is applied after the nonlinearity, never as -inf before it, as "HSTU
-// tensor by tensor: SiLU aggregation, temporal bias and gating", section "Do not copy softmax
-// masking mechanically", requires), round it to bf16 into shared memory, and tcgen05 adds
-// A V into the fp32 output accumulator in TMEM.  The 1/N scale ("HSTU-MUSA: HSTU for Moore
-// Threads (MUSA)", "Accuracy Alignment": N = batch max_seqlen) is applied once to the
-// accumulator, and Y goes to global memory in fp32 for the LayerNorm + gating kernel.
+// One CTA per (128-row query tile, sequence, head).  For every key tile of 128 that holds a
+// valid pair:  S = Q K^T on tcgen05 (bf16 operands staged by TMA in 128-byte-swizzled shared
+// memory, fp32 accumulator in TMEM); the epilogue warps read S from TMEM and form
+// A = mask ? SiLU(alpha*S + b) : 0 in fp32, where b is the relative-position plus bucketed
+// time bias and the mask is applied after the nonlinearity, never as -inf before it ("HSTU
+// tensor by tensor: SiLU aggregation, temporal bias and gating", sections "Similar shape,
+// different aggregation" and "Do not copy softmax masking mechanically"); A is rounded to
+// bf16 and written back over S in TMEM (two elements per 32-bit column), and tcgen05 adds
+// A V into the fp32 output accumulator in TMEM with A read from TMEM.  The 1/N scale
+// ("HSTU-MUSA: HSTU for Moore Threads (MUSA)", "Accuracy Alignment": N = batch max_seqlen)
+// is applied once to the accumulator; Y goes to global memory in fp32.
 //
-// Warp roles: warp 0 lane 0 issues TMA loads (Q once, K/V double-buffered), warp 1 lane 0
-// issues the MMAs, warp 2 owns the TMEM allocation, warps 4-7 are the epilogue (one query
-// row per thread, which is also the row's TMEM lane).  S is double-buffered in TMEM so
-// QK^T of the next tile runs while the epilogue works on the current one.  Every wait is
-// bounded; a timeout sets HSTU_DEV_WAIT_TIMEOUT and the CTA unwinds.
+// Warp roles (12 warps): warp 0 lane 0 issues TMA loads (Q once, K/V double-buffered);
+// warp 1 lane 0 issues the MMAs; warp 2 owns TMEM; warp 3 stages each key tile's timestamps
+// and their range; warps 4-7 and 8-11 are two epilogue warpgroups, each owning 64 of the
+// 128 key columns of every query row (thread = row = TMEM lane).  S is double-buffered, so
+// QK^T of the next tile runs while the epilogue works on this one.
+//
+// Bias evaluation per (row, 64-key half tile):  the time bucket is computed once for the
+// smallest and largest |dt| the half can produce (from the half's timestamp range); when
+// both agree (the common case away from the diagonal) the time bias is a per-row constant.
+// The rel index runs p(i)-j down a contiguous window of the table when no clamping occurs.
+// Mask evaluation is skipped on tiles the mask covers fully.  Every wait is bounded; a
+// timeout sets HSTU_DEV_WAIT_TIMEOUT and the CTA unwinds.
 #include <cudaTypedefs.h>
 
 #include <cstring>
@@ -29,28 +37,58 @@ using namespace sm100;
 
 namespace {
 
-constexpr int BM = 128, BN = 128;
-constexpr int kTcThreads = 256;
+constexpr int BM = 128, BN = 128, HALF = 64;
+constexpr int kTcThreads = 384;
 constexpr int kRelSmemMax = 4096;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kBlockBytes = 128 * 128;   // one 128-row x 64-element bf16 swizzle block
+constexpr uint32_t kOCol = 256;          // TMEM column of the output accumulator
 
 enum Bar { Q_FULL = 0, KV_FULL = 1, KV_EMPTY = 3, S_FULL = 5, S_FREE = 7, P_FULL = 9,
-           P_FREE = 10, O_FULL = 11, MMA_DONE = 12, NUM_BARS = 13 };
+           META_FULL = 11, O_FULL = 13, MMA_DONE = 14, NUM_BARS = 15 };
+
+struct TileMeta {
+    int64_t tmin[2], tmax[2];   // timestamp range of each 64-key half (valid keys only)
+    int32_t ok32[2];            // the half's range is below 2^31 - 1: 32-bit relative stamps valid
+    int32_t pad[2];
+};
+
+// Exact time-bucket lookup on y = |dt| + 1 < 2^31: cell q = 32*floor(log2 y) + (next 5 bits of
+// y), i.e. the top bits of y's float representation.  A cell spans less than 1/32 of its
+// value while distinct bucket thresholds differ by a larger factor (checked when the
+// table is built), so at most one distinct threshold falls inside a cell:
+//   bucket(dt) = base + (dt >= next ? jump : 0).
+struct LutEntry {
+    uint32_t next;   // the threshold inside the cell (UINT32_MAX: none)
+    int16_t base;    // bucket of the cell's smallest |dt|
+    int16_t jump;    // thresholds equal to `next` (buckets gained at it)
+};
+constexpr int kLutCells = 1024;
+
+__device__ __forceinline__ int lut_cell(uint32_t dt)
+{
+    const uint32_t y = dt + 1u;
+    const bool big = y >= (1u << 23);
+    const uint32_t ys = big ? (y >> 8) : y;                 // < 2^23: exact in fp32
+    const float f = __uint_as_float(0x4B000000u | ys) - 8388608.0f;
+    return (int)(__float_as_uint(f) >> 18) - (127 << 5) + (big ? (8 << 5) : 0);
+}
 
 template <int DQK, int DV>
 struct FwdLayout {
     static constexpr int QB = BM * DQK * 2;
     static constexpr int KB = BN * DQK * 2;
     static constexpr int VB = BN * DV * 2;
-    static constexpr int PB = BM * BN * 2;
     static constexpr int Q_OFF = 0;
     static constexpr int K_OFF = Q_OFF + QB;
     static constexpr int V_OFF = K_OFF + 2 * KB;
-    static constexpr int P_OFF = V_OFF + 2 * VB;
-    static constexpr int BAR_OFF = P_OFF + PB;
+    static constexpr int BAR_OFF = V_OFF + 2 * VB;
     static constexpr int SLOT_OFF = BAR_OFF + 8 * 16;
-    static constexpr int THR_OFF = SLOT_OFF + 16;
+    static constexpr int META_OFF = SLOT_OFF + 16;
+    static constexpr int TSK_OFF = META_OFF + 2 * (int)sizeof(TileMeta);
+    static constexpr int TSK32_OFF = TSK_OFF + 2 * BN * 8;
+    static constexpr int LUT_OFF = TSK32_OFF + 2 * BN * 4;
+    static constexpr int THR_OFF = LUT_OFF + kLutCells * 8;
     static constexpr int TB_OFF = THR_OFF + 8 * kMaxTimeBuckets;
     static constexpr int REL_OFF = TB_OFF + 4 * kMaxTimeBuckets;
     static constexpr int TOTAL = REL_OFF + 4 * kRelSmemMax;
@@ -77,10 +115,88 @@ struct TileIter {
     }
 };
 
-__device__ __forceinline__ void report_timeout(const DevParams &p) { flag_error(p, HSTU_DEV_WAIT_TIMEOUT); }
+__device__ __forceinline__ void report_timeout(const DevParams &p)
+{
+    flag_error(p, HSTU_DEV_WAIT_TIMEOUT);
+}
+
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity)
+{
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity));
+}
+
+// Bucket of dt known to lie in [lo, hi]: number of thresholds <= dt (thr[k-1] opens bucket k).
+__device__ __forceinline__ int bucket_in(const uint64_t *thr, int lo, int hi, uint64_t dt)
+{
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (thr[mid - 1] <= dt) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+// Keys [a, b] intersected with [jh, jh+63], as bits relative to jh.
+__device__ __forceinline__ uint64_t range_bits(int a, int b, int jh)
+{
+    const int lo = max(a, jh) - jh, hi = min(b, jh + HALF - 1) - jh;
+    if (lo > hi) return 0ull;
+    const int n = hi - lo + 1;
+    const uint64_t m = n >= 64 ? ~0ull : ((1ull << n) - 1ull);
+    return m << lo;
+}
+
+// Valid keys of row i among [jh, jh+63] (bit c <-> key jh + c): the contextual prefix for
+// every row; for non-contextual rows the causal (windowed) history keys up to p(i); for a
+// candidate row also itself.  Equivalent to pair_valid over the half tile.
+__device__ __forceinline__ uint64_t row_valid_bits(int i, int jh, const SeqInfo &s, int W)
+{
+    if (i >= s.L) return 0ull;
+    uint64_t m = range_bits(0, s.c - 1, jh);
+    if (i < s.c) return m;
+    const int pi = clamp_pos(i, s.E);
+    const int lo = W > 0 ? max(s.c, pi - W) : s.c;
+    m |= range_bits(lo, min(pi, s.E - 1), jh);
+    if (i >= s.E) m |= range_bits(i, i, jh);
+    return m;
+}
+
+// Fills the time-bucket lookup table; clears *valid when some cell holds two thresholds
+// (bucket thresholds closer than the cell resolution), which disables the table.
+__device__ void build_lut(const uint64_t *thr, int n_thr, LutEntry *lut, int32_t *valid)
+{
+    for (int q = threadIdx.x; q < kLutCells; q += blockDim.x) {
+        const int e = q >> 5, m = q & 31;
+        const uint64_t ylo = (((uint64_t)(32 + m) << e) + 31) >> 5;      // ceil(2^e (32+m)/32)
+        const uint64_t yhi = ((((uint64_t)(33 + m) << e) + 31) >> 5) - 1; // last y in the cell
+        LutEntry ent;
+        ent.next = 0xFFFFFFFFu;
+        ent.base = 0;
+        ent.jump = 0;
+        if (ylo >= 1 && ylo <= yhi) {
+            const uint64_t dlo = ylo - 1, dhi = yhi - 1;
+            const int b = bucket_search(thr, n_thr, dlo);
+            ent.base = (int16_t)b;
+            if (b < n_thr && thr[b] <= dhi) {
+                int n = 1;
+                while (b + n < n_thr && thr[b + n] == thr[b]) ++n;
+                if (b + n < n_thr && thr[b + n] <= dhi) atomicAnd(valid, 0);
+                if (thr[b] > 0xFFFFFFFEull) atomicAnd(valid, 0);
+                ent.next = (uint32_t)min(thr[b], (uint64_t)0xFFFFFFFEull);
+                ent.jump = (int16_t)n;
+            }
+        }
+        lut[q] = ent;
+    }
+}
+
+__device__ __forceinline__ int64_t shfl_xor_i64(int64_t v, int m)
+{
+    return (int64_t)__shfl_xor_sync(0xffffffffu, (long long)v, m);
+}
 
 template <int DQK, int DV>
-__global__ void __launch_bounds__(kTcThreads, 1) fwd_tc_kernel(const __grid_constant__ FwdTcArgs args)
+__global__ void __launch_bounds__(kTcThreads, 1)
+    fwd_tc_kernel(const __grid_constant__ FwdTcArgs args)
 {
     using L = FwdLayout<DQK, DV>;
     const DevParams &p = args.p;
@@ -94,6 +210,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) fwd_tc_kernel(const __grid_cons
                                               ~static_cast<uintptr_t>(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::BAR_OFF);
     uint32_t *slot = reinterpret_cast<uint32_t *>(sm + L::SLOT_OFF);
+    TileMeta *meta = reinterpret_cast<TileMeta *>(sm + L::META_OFF);
+    int64_t *tsk = reinterpret_cast<int64_t *>(sm + L::TSK_OFF);
+    int32_t *tsk32 = reinterpret_cast<int32_t *>(sm + L::TSK32_OFF);
+    LutEntry *lutp = reinterpret_cast<LutEntry *>(sm + L::LUT_OFF);
+    int32_t *lut_valid = reinterpret_cast<int32_t *>(sm + L::SLOT_OFF + 4);
     uint64_t *thr = reinterpret_cast<uint64_t *>(sm + L::THR_OFF);
     float *tbs = reinterpret_cast<float *>(sm + L::TB_OFF);
     float *rels = reinterpret_cast<float *>(sm + L::REL_OFF);
@@ -105,10 +226,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) fwd_tc_kernel(const __grid_cons
             mbar_init(&bars[KV_FULL + x], 1);
             mbar_init(&bars[KV_EMPTY + x], 1);
             mbar_init(&bars[S_FULL + x], 1);
-            mbar_init(&bars[S_FREE + x], 128);
+            mbar_init(&bars[S_FREE + x], 1);
+            mbar_init(&bars[P_FULL + x], 256);
+            mbar_init(&bars[META_FULL + x], 32);
         }
-        mbar_init(&bars[P_FULL], 128);
-        mbar_init(&bars[P_FREE], 1);
         mbar_init(&bars[O_FULL], 1);
         mbar_init(&bars[MMA_DONE], 1);
         fence_mbar_init();
@@ -119,6 +240,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) fwd_tc_kernel(const __grid_cons
     const bool rel_in_smem = p.R <= kRelSmemMax;
     if (rel_in_smem)
         for (int x = threadIdx.x; x < p.R; x += kTcThreads) rels[x] = p.rel[x];
+    if (threadIdx.x == 0) *lut_valid = 1;
+    __syncthreads();
+    if (p.NB > 0) build_lut(thr, p.n_thr, lutp, lut_valid);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -156,7 +280,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) fwd_tc_kernel(const __grid_cons
                 ++it;
             }
             if (!ok) report_timeout(p);
-            // Loads issued must land before the CTA can exit (bounded).
+            // loads issued must land before the CTA exits (bounded)
             bool drained = mbar_wait(&bars[Q_FULL], 0);
             for (int x = it - 1; x >= 0 && x >= it - 2; --x)
                 drained &= mbar_wait(&bars[KV_FULL + (x & 1)], (x >> 1) & 1);
@@ -168,23 +292,22 @@ __global__ void __launch_bounds__(kTcThreads, 1) fwd_tc_kernel(const __grid_cons
             constexpr uint32_t idesc_qk = idesc_bf16(BM, BN, false, false);
             constexpr uint32_t idesc_pv = idesc_bf16(BM, DV, false, true);
             const uint32_t q_addr = sm_base + L::Q_OFF;
-            const uint32_t p_addr = sm_base + L::P_OFF;
-            const uint32_t o_tmem = tmem + 256;
             bool ok = mbar_wait(&bars[Q_FULL], 0);
             tc_fence_after();
             auto issue_pv = [&](int x) -> bool {
-                if (!mbar_wait(&bars[P_FULL], x & 1)) return false;
+                const int sx = x & 1;
+                if (!mbar_wait(&bars[P_FULL + sx], (x >> 1) & 1)) return false;
                 tc_fence_after();
-                const uint32_t v_addr = sm_base + L::V_OFF + (x & 1) * L::VB;
+                const uint32_t v_addr = sm_base + L::V_OFF + sx * L::VB;
 #pragma unroll
                 for (int kk = 0; kk < BN / 16; ++kk) {
-                    const uint64_t a = sw128_desc(p_addr + (kk >> 2) * kBlockBytes + (kk & 3) * 32,
-                                                  16, 1024);
+                    // keys 16kk..16kk+15: half (kk/4) packed at columns [64*half, 64*half+32)
+                    const uint32_t a_tmem = tmem + sx * 128 + (kk >> 2) * 64 + (kk & 3) * 8;
                     const uint64_t bd = sw128_desc(v_addr + kk * 2048, kBlockBytes, 1024);
-                    umma_bf16_ss(o_tmem, a, bd, idesc_pv, (x > 0 || kk > 0) ? 1u : 0u);
+                    umma_bf16_ts(tmem + kOCol, a_tmem, bd, idesc_pv, (x > 0 || kk > 0) ? 1u : 0u);
                 }
-                umma_commit(&bars[P_FREE]);
-                umma_commit(&bars[KV_EMPTY + (x & 1)]);
+                umma_commit(&bars[S_FREE + sx]);
+                umma_commit(&bars[KV_EMPTY + sx]);
                 return true;
             };
             TileIter t(s, i0, p.W);
@@ -198,14 +321,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) fwd_tc_kernel(const __grid_cons
                 }
                 tc_fence_after();
                 const uint32_t k_addr = sm_base + L::K_OFF + st * L::KB;
-                const uint32_t s_tmem = tmem + st * 128;
 #pragma unroll
                 for (int kb = 0; kb < DQK / 64; ++kb)
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks) {
                         const uint64_t a = sw128_desc(q_addr + kb * kBlockBytes + ks * 32, 16, 1024);
                         const uint64_t bd = sw128_desc(k_addr + kb * kBlockBytes + ks * 32, 16, 1024);
-                        umma_bf16_ss(s_tmem, a, bd, idesc_qk, (kb | ks) ? 1u : 0u);
+                        umma_bf16_ss(tmem + st * 128, a, bd, idesc_qk, (kb | ks) ? 1u : 0u);
                     }
                 umma_commit(&bars[S_FULL + st]);
                 if (it >= 1 && !issue_pv(it - 1)) { ok = false; break; }
@@ -218,95 +340,234 @@ __global__ void __launch_bounds__(kTcThreads, 1) fwd_tc_kernel(const __grid_cons
             umma_commit(&bars[MMA_DONE]);
             if (!mbar_wait(&bars[MMA_DONE], 0)) report_timeout(p);
         }
+    } else if (warp == 3) {
+        // -------------------------------------------------------------------- tile metadata
+        const bool use_ts = p.NB > 0;
+        TileIter t(s, i0, p.W);
+        int it = 0;
+        while (t.next()) {
+            const int st = it & 1;
+            if (it >= 2 && !warp_wait(&bars[S_FREE + st], ((it >> 1) - 1) & 1)) {
+                report_timeout(p);
+                break;
+            }
+            if (use_ts) {
+                const int j0 = t.kt * BN;
+                int64_t v[4];
+                int64_t mn[2] = {INT64_MAX, INT64_MAX}, mx[2] = {INT64_MIN, INT64_MIN};
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    const int c = lane + 32 * q4;
+                    const int j = j0 + c;
+                    v[q4] = 0;
+                    if (j < s.L) {
+                        v[q4] = p.ts[s.start + clamp_pos(j, s.E)];
+                        mn[q4 >> 1] = min(mn[q4 >> 1], v[q4]);
+                        mx[q4 >> 1] = max(mx[q4 >> 1], v[q4]);
+                    }
+                }
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) {
+                        mn[hh] = min(mn[hh], shfl_xor_i64(mn[hh], o));
+                        mx[hh] = max(mx[hh], shfl_xor_i64(mx[hh], o));
+                    }
+                }
+                int ok32[2];
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh)
+                    ok32[hh] = mn[hh] > mx[hh] ||
+                               (uint64_t)mx[hh] - (uint64_t)mn[hh] < (uint64_t)INT32_MAX;
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    const int c = lane + 32 * q4, hh = q4 >> 1;
+                    tsk[st * BN + c] = v[q4];
+                    // stamps relative to the half's minimum (0 for keys past the sequence)
+                    const int j = j0 + c;
+                    tsk32[st * BN + c] =
+                        (j < s.L && ok32[hh]) ? (int32_t)((uint64_t)v[q4] - (uint64_t)mn[hh]) : 0;
+                }
+                if (lane == 0) {
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        meta[st].tmin[hh] = mn[hh];
+                        meta[st].tmax[hh] = mx[hh];
+                        meta[st].ok32[hh] = ok32[hh];
+                    }
+                }
+            }
+            __syncwarp();
+            mbar_arrive(&bars[META_FULL + st]);
+            ++it;
+        }
     } else if (warp >= 4) {
         // -------------------------------------------------------------------- epilogue
-        const int r = threadIdx.x - 128;            // query row in the tile == TMEM lane
+        const int wg = (warp - 4) >> 2;               // 0: keys 0..63, 1: keys 64..127
+        const int r = (warp & 3) * 32 + lane;         // query row in the tile == TMEM lane
         const int i = i0 + r;
+        const bool row_in = i < s.L;
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
         const int pi = clamp_pos(i, s.E);
         const bool use_ts = p.NB > 0;
-        const int64_t tsi = (use_ts && i < s.L) ? p.ts[s.start + pi] : 0;
-        const int64_t *tsg = p.ts + s.start;
+        const bool use_rel = p.R > 0;
+        const int64_t tsi = (use_ts && row_in) ? p.ts[s.start + pi] : 0;
         const float *relp = rel_in_smem ? rels : p.rel;
         const float half_alpha = 0.5f * p.alpha;
-        const uint32_t p_row = sm_base + L::P_OFF + r * 128;
+        const bool lut_ok = *lut_valid != 0;
         bool ok = true;
         TileIter t(s, i0, p.W);
         int it = 0;
         while (t.next()) {
             const int st = it & 1;
-            const int j0 = t.kt * BN;
-            const bool full = tile_all_valid(i0, i0 + BM - 1, j0, j0 + BN - 1, s, p.W);
-            // warp-uniform outcome, so the .sync.aligned TMEM loads below never diverge
-            if (!__all_sync(0xffffffffu, mbar_wait(&bars[S_FULL + st], (it >> 1) & 1))) {
+            const int jh = t.kt * BN + wg * HALF;     // first key of this warpgroup's half
+            const bool full = tile_all_valid(i0, i0 + BM - 1, jh, jh + HALF - 1, s, p.W);
+            if (!warp_wait(&bars[META_FULL + st], (it >> 1) & 1) ||
+                !warp_wait(&bars[S_FULL + st], (it >> 1) & 1)) {
                 ok = false;
                 break;
             }
-            if (it >= 1 && !__all_sync(0xffffffffu, mbar_wait(&bars[P_FREE], (it - 1) & 1))) {
-                ok = false;
-                break;
+
+            // ---- per (row, half tile) structure; path choices are made warp-uniform
+            const uint64_t vmask = full ? ~0ull : row_valid_bits(i, jh, s, p.W);
+            const int rbase = pi - jh;                // rel index of key jh + c is rbase - c
+            const bool rdirect = __all_sync(0xffffffffu, !use_rel || (rbase - (HALF - 1) >= 0 &&
+                                                                        rbase <= p.R - 1));
+            // time bias: tmode 0 = per-row constant, 1 = one bucket boundary (compare in
+            // 32-bit relative stamps), 2 = exact lookup table, 3 = 64-bit search
+            int tmode = 0;
+            float tb_lo = 0.f, tb_hi = 0.f;
+            int32_t cmpA = INT32_MIN, cmpB = INT32_MAX, tsi_rel = 0;
+            int blo = 0, bhi = 0;
+            bool lane_const = true;
+            if (use_ts) {
+                const int64_t hmin = meta[st].tmin[wg], hmax = meta[st].tmax[wg];
+                const bool h32 = meta[st].ok32[wg] != 0;
+                int my_mode = 0;
+                if (row_in && hmin <= hmax) {
+                    uint64_t dlo, dhi;
+                    if (tsi >= hmax) {
+                        dlo = (uint64_t)tsi - (uint64_t)hmax;
+                        dhi = (uint64_t)tsi - (uint64_t)hmin;
+                    } else if (tsi <= hmin) {
+                        dlo = (uint64_t)hmin - (uint64_t)tsi;
+                        dhi = (uint64_t)hmax - (uint64_t)tsi;
+                    } else {
+                        dlo = 0;
+                        const uint64_t a = (uint64_t)tsi - (uint64_t)hmin;
+                        const uint64_t c = (uint64_t)hmax - (uint64_t)tsi;
+                        dhi = a > c ? a : c;
+                    }
+                    blo = bucket_in(thr, 0, p.n_thr, dlo);
+                    bhi = bucket_in(thr, blo, p.n_thr, dhi);
+                    const bool fits = h32 && dhi < (uint64_t)(INT32_MAX - 1);
+                    if (fits) tsi_rel = (int32_t)((uint64_t)tsi - (uint64_t)hmin);
+                    if (bhi == blo) {
+                        my_mode = 0;
+                    } else if (bhi == blo + 1 && fits) {
+                        my_mode = 1;
+                        // |tsi - tsj| >= T  <=>  tsj <= tsi - T  or  tsj >= tsi + T
+                        const int64_t T = (int64_t)thr[blo];
+                        const int64_t A = (int64_t)tsi_rel - T, B = (int64_t)tsi_rel + T;
+                        cmpA = (int32_t)max((int64_t)INT32_MIN, min((int64_t)INT32_MAX, A));
+                        cmpB = (int32_t)max((int64_t)INT32_MIN, min((int64_t)INT32_MAX, B));
+                    } else {
+                        my_mode = (fits && lut_ok) ? 2 : 3;
+                    }
+                }
+                lane_const = my_mode == 0;
+                tmode = __reduce_max_sync(0xffffffffu, my_mode);
+                tb_lo = tbs[blo];
+                tb_hi = tbs[min(blo + 1, p.NB - 1)];
             }
+            const int32_t *tk32 = tsk32 + st * BN + wg * HALF;
+            const int64_t *tk64 = tsk + st * BN + wg * HALF;
+
             tc_fence_after();
 #pragma unroll 1
-            for (int half = 0; half < 2; ++half) {
-                uint32_t ra[32], rb[32];
-                tmem_ld32(tmem + lane_base + st * 128 + half * 64, ra);
-                tmem_ld32(tmem + lane_base + st * 128 + half * 64 + 32, rb);
+            for (int ch = 0; ch < 2; ++ch) {
+                const uint32_t s_col = tmem + lane_base + st * 128 + wg * HALF + ch * 32;
+                uint32_t ra[32];
+                tmem_ld32(s_col, ra);
                 tmem_wait_ld();
                 reg_fence(ra);
-                reg_fence(rb);
-                uint32_t pk[32];
+                const uint32_t vbits = (uint32_t)(vmask >> (32 * ch));
+                const int cb = ch * 32;
+                float av[32];
+                // bias: rel part
 #pragma unroll
-                for (int c2 = 0; c2 < 32; ++c2) {
-                    float av[2];
+                for (int c = 0; c < 32; ++c) {
+                    float bias = 0.f;
+                    if (use_rel) {
+                        if (rdirect) {
+                            bias = relp[rbase - cb - c];
+                        } else {
+                            int ri = rbase - cb - c;
+                            ri = ri < 0 ? 0 : (ri > p.R - 1 ? p.R - 1 : ri);
+                            bias = relp[ri];
+                        }
+                    }
+                    av[c] = bias;
+                }
+                // bias: time part
+                if (tmode == 0) {
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) av[c] += tb_lo;
+                } else if (tmode == 1) {
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) {
+                        const int32_t tj = tk32[cb + c];
+                        av[c] += (tj <= cmpA || tj >= cmpB) ? tb_hi : tb_lo;
+                    }
+                } else if (tmode == 2) {
+                    const LutEntry *lut = reinterpret_cast<const LutEntry *>(lutp);
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) {
+                        int32_t d = tsi_rel - tk32[cb + c];
+                        uint32_t dt = (uint32_t)(d < 0 ? -d : d);
+                        dt = min(dt, (uint32_t)INT32_MAX - 1u);
+                        const LutEntry e = lut[lut_cell(dt)];
+                        const float v = tbs[e.base + (dt >= e.next ? e.jump : 0)];
+                        av[c] += lane_const ? tb_lo : v;
+                    }
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 32; ++c)
+                        av[c] += tbs[bucket_search(thr, p.n_thr, abs_diff_u64(tsi, tk64[cb + c]))];
+                }
+                // SiLU(x) = x sigmoid(x) = h + h tanh(h), h = x/2; mask after the nonlinearity
+                uint32_t pk[16];
+#pragma unroll
+                for (int c2 = 0; c2 < 16; ++c2) {
+                    float a2[2];
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
-                        const int c = 2 * c2 + e;                 // column within the half
-                        const int j = j0 + half * 64 + c;
-                        const uint32_t raw = c < 32 ? ra[c] : rb[c - 32];
-                        const bool valid = full || (i < s.L && j < s.L && pair_valid(i, j, s, p.W));
-                        float bias = 0.f;
-                        const int pj = clamp_pos(j, s.E);
-                        if (p.R > 0) {
-                            int ri = pi - pj;
-                            ri = ri < 0 ? 0 : (ri > p.R - 1 ? p.R - 1 : ri);
-                            bias += relp[ri];
-                        }
-                        if (use_ts) {
-                            const int64_t tsj = j < s.L ? __ldg(tsg + pj) : 0;
-                            bias += tbs[bucket_search(thr, p.n_thr, abs_diff_u64(tsi, tsj))];
-                        }
-                        // SiLU(x) = x*sigmoid(x) = h + h*tanh(h) with h = x/2
-                        const float hx = fmaf(half_alpha, __uint_as_float(raw), 0.5f * bias);
+                        const int c = 2 * c2 + e;
+                        const float hx = fmaf(half_alpha, __uint_as_float(ra[c]), 0.5f * av[c]);
                         const float a = fmaf(hx, tanh_approx(hx), hx);
-                        av[e] = valid ? a : 0.f;
+                        a2[e] = full ? a : (((vbits >> c) & 1u) ? a : 0.f);
                     }
-                    pk[c2] = pack_bf16x2(av[0], av[1]);
+                    pk[c2] = pack_bf16x2(a2[0], a2[1]);
                 }
-                // 128-byte-swizzled K-major A operand: 16-byte chunk ch of row r at (ch ^ (r&7))
-                const uint32_t blk = p_row + half * kBlockBytes;
-#pragma unroll
-                for (int ch = 0; ch < 8; ++ch)
-                    st_shared_v4(blk + ((ch ^ (r & 7)) << 4), pk[4 * ch], pk[4 * ch + 1],
-                                 pk[4 * ch + 2], pk[4 * ch + 3]);
+                // bf16 A over the first 32 of this warpgroup's 64 S columns
+                tmem_st16(tmem + lane_base + st * 128 + wg * HALF + ch * 16, pk);
             }
+            tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(&bars[S_FREE + st]);
-            fence_proxy_async_smem();
-            mbar_arrive(&bars[P_FULL]);
+            mbar_arrive(&bars[P_FULL + st]);
             ++it;
         }
-        if (ok && !__all_sync(0xffffffffu, mbar_wait(&bars[O_FULL], 0))) ok = false;
+        if (ok && !warp_wait(&bars[O_FULL], 0)) ok = false;
         if (ok) {
             tc_fence_after();
             float *yr = args.y + (s.start + i) * (int64_t)p.D + h * DV;
 #pragma unroll 1
-            for (int c = 0; c < DV / 32; ++c) {
+            for (int c = wg * (DV / 64); c < (wg + 1) * (DV / 64); ++c) {
                 uint32_t ra[32];
-                tmem_ld32(tmem + lane_base + 256 + c * 32, ra);
+                tmem_ld32(tmem + lane_base + kOCol + c * 32, ra);
                 tmem_wait_ld();
                 reg_fence(ra);
-                if (i < s.L) {
+                if (row_in) {
                     float4 *dst = reinterpret_cast<float4 *>(yr + c * 32);
 #pragma unroll
                     for (int x = 0; x < 8; ++x)
@@ -363,7 +624,8 @@ cudaError_t launch_tc(const FwdTcArgs &a, cudaStream_t st)
 {
     using L = FwdLayout<DQK, DV>;
     auto kern = fwd_tc_kernel<DQK, DV>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
     if (e != cudaSuccess) return e;
     dim3 grid((a.p.N + BM - 1) / BM, a.p.B, a.p.H);
     kern<<<grid, kTcThreads, L::ALLOC, st>>>(a);
