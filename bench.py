@@ -16,7 +16,6 @@ import argparse
 import json
 import os
 import statistics
-import subprocess
 import sys
 import time
 
@@ -50,53 +49,62 @@ def dist_setup(args):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms during the timed region."""
-    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clocks and clock-event (throttle) reasons polled through NVML every few ms while
+    the timed region runs (read-only queries)."""
+    REASONS = {"hw_slowdown": "nvmlClocksEventReasonHwSlowdown",
+               "hw_thermal_slowdown": "nvmlClocksEventReasonHwThermalSlowdown",
+               "sw_thermal_slowdown": "nvmlClocksEventReasonSwThermalSlowdown",
+               "sw_power_cap": "nvmlClocksEventReasonSwPowerCap",
+               "hw_power_brake": "nvmlClocksEventReasonHwPowerBrakeSlowdown"}
 
-    def __init__(self, gpu_index):
+    def __init__(self, gpu_index, period_s=0.002):
         self.gpu = gpu_index
-        self.proc = None
-        self.path = os.path.join("/tmp", "hstu_clocks_%d_%d.csv" % (os.getpid(), gpu_index))
+        self.bus_id = None
+        try:
+            import torch
+            pr = torch.cuda.get_device_properties(gpu_index)
+            self.bus_id = "%08x:%02x:%02x.0" % (pr.pci_domain_id, pr.pci_bus_id, pr.pci_device_id)
+        except Exception:
+            pass
+        self.period = period_s
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.err = None
+
+    def _run(self):
+        import pynvml
+        try:
+            pynvml.nvmlInit()
+            hd = (pynvml.nvmlDeviceGetHandleByPciBusId(self.bus_id) if self.bus_id
+                  else pynvml.nvmlDeviceGetHandleByIndex(self.gpu))
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(hd, pynvml.NVML_CLOCK_SM)
+            masks = {k: getattr(pynvml, v, 0) for k, v in self.REASONS.items()}
+            while not self.stop_flag.is_set():
+                self.samples.append(pynvml.nvmlDeviceGetClockInfo(hd, pynvml.NVML_CLOCK_SM))
+                r = pynvml.nvmlDeviceGetCurrentClocksEventReasons(hd)
+                for k, m in masks.items():
+                    if m and (r & m):
+                        self.reasons.add(k)
+                time.sleep(self.period)
+            pynvml.nvmlShutdown()
+        except Exception as e:  # NVML unavailable: report it instead of clocks
+            self.err = repr(e)
 
     def start(self):
-        try:
-            self.f = open(self.path, "w")
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.QUERY,
-                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
-                stderr=subprocess.DEVNULL)
-        except OSError:
-            self.proc = None
+        import threading
+        self.stop_flag = threading.Event()
+        self.th = threading.Thread(target=self._run, daemon=True)
+        self.th.start()
+        time.sleep(0.02)
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        self.f.close()
-        sm, smax, reasons = [], None, set()
-        names = ["active", "hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
-                 "sw_power_cap"]
-        for line in open(self.path):
-            parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                smax = float(parts[2])
-            except ValueError:
-                continue
-            for name, val in zip(names[1:], parts[5:9]):
-                if val.lower() in ("active", "1", "yes"):
-                    reasons.add(name)
-        os.unlink(self.path)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        self.stop_flag.set()
+        self.th.join(timeout=5)
+        if self.err or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz,
+                    "reasons": ["nvml unavailable: %s" % self.err] if self.err else [],
+                    "samples": len(self.samples)}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
 def stage_timer(ops, torch, stages):

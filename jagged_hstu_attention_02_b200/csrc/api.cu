@@ -245,7 +245,7 @@ hstu_status_t hstu_attn_fwd(const hstu_attn_params_t *p, const void *q, const vo
         if (p->dtype == HSTU_F32)
             HSTU_CUDA_TRY(launch_simt_fwd<float>(d, q, k, v, y, s));
         else if (tc_fwd_supported(p->d_qk, p->d_v, p->total_tokens))
-            HSTU_CUDA_TRY(launch_tc_fwd(d, q, k, v, y, s));
+            HSTU_CUDA_TRY(launch_tc_fwd(d, q, k, v, y, train, s));
         else
             HSTU_CUDA_TRY(launch_simt_fwd<__nv_bfloat16>(d, q, k, v, y, s));
     }
@@ -298,22 +298,27 @@ hstu_status_t hstu_attn_bwd(const hstu_attn_params_t *p, const void *dout, const
     ws += align_up((size_t)p->total_tokens * p->num_heads * p->d_v * 4, 256);
     const int64_t nq = p->total_tokens * p->num_heads * p->d_qk;
     const bool f32 = p->dtype == HSTU_F32;
+    const bool tc = !f32 && tc_bwd_supported(p->d_qk, p->d_v, p->total_tokens);
     float *dq_acc = f32 ? reinterpret_cast<float *>(dq) : reinterpret_cast<float *>(ws);
     HSTU_CUDA_TRY(cudaMemsetAsync(dq_acc, 0, sizeof(float) * nq, s));
     {
         StageScope scope(HSTU_STAGE_BWD_NORM, s);
         if (f32)
             HSTU_CUDA_TRY(launch_ln_gate_bwd<float>(d, dout, u, saved_y, saved_mean, saved_rstd,
-                                                    du, dy, s));
+                                                    du, dy, false, s));
         else
             HSTU_CUDA_TRY(launch_ln_gate_bwd<__nv_bfloat16>(d, dout, u, saved_y, saved_mean,
-                                                            saved_rstd, du, dy, s));
+                                                            saved_rstd, du, dy, tc, s));
     }
     {
         StageScope scope(HSTU_STAGE_BWD_ATTN, s);
         if (f32) {
             HSTU_CUDA_TRY(launch_simt_bwd<float>(d, q, k, v, dy, dq_acc, dk, dv, d_rel_bias,
                                                  d_time_bias, s));
+        } else if (tc) {
+            HSTU_CUDA_TRY(launch_tc_bwd(d, q, k, v, dy, dq_acc, dk, dv, d_rel_bias, d_time_bias,
+                                        s));
+            HSTU_CUDA_TRY(launch_convert<__nv_bfloat16>(dq_acc, dq, nq, s));
         } else {
             HSTU_CUDA_TRY(launch_simt_bwd<__nv_bfloat16>(d, q, k, v, dy, dq_acc, dk, dv,
                                                          d_rel_bias, d_time_bias, s));

@@ -28,6 +28,7 @@
 
 #include <cstring>
 
+#include "bias.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -37,7 +38,7 @@ using namespace sm100;
 
 namespace {
 
-constexpr int BM = 128, BN = 128, HALF = 64;
+constexpr int BM = 128, BN = 128, HALF = kHalf;
 constexpr int kTcThreads = 384;
 constexpr int kRelSmemMax = 4096;
 constexpr uint32_t kTmemCols = 512;
@@ -52,27 +53,6 @@ struct TileMeta {
     int32_t ok32[2];            // the half's range is below 2^31 - 1: 32-bit relative stamps valid
     int32_t pad[2];
 };
-
-// Exact time-bucket lookup on y = |dt| + 1 < 2^31: cell q = 32*floor(log2 y) + (next 5 bits of
-// y), i.e. the top bits of y's float representation.  A cell spans less than 1/32 of its
-// value while distinct bucket thresholds differ by a larger factor (checked when the
-// table is built), so at most one distinct threshold falls inside a cell:
-//   bucket(dt) = base + (dt >= next ? jump : 0).
-struct LutEntry {
-    uint32_t next;   // the threshold inside the cell (UINT32_MAX: none)
-    int16_t base;    // bucket of the cell's smallest |dt|
-    int16_t jump;    // thresholds equal to `next` (buckets gained at it)
-};
-constexpr int kLutCells = 1024;
-
-__device__ __forceinline__ int lut_cell(uint32_t dt)
-{
-    const uint32_t y = dt + 1u;
-    const bool big = y >= (1u << 23);
-    const uint32_t ys = big ? (y >> 8) : y;                 // < 2^23: exact in fp32
-    const float f = __uint_as_float(0x4B000000u | ys) - 8388608.0f;
-    return (int)(__float_as_uint(f) >> 18) - (127 << 5) + (big ? (8 << 5) : 0);
-}
 
 template <int DQK, int DV>
 struct FwdLayout {
@@ -125,76 +105,10 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity)
     return __all_sync(0xffffffffu, mbar_wait(bar, parity));
 }
 
-// Bucket of dt known to lie in [lo, hi]: number of thresholds <= dt (thr[k-1] opens bucket k).
-__device__ __forceinline__ int bucket_in(const uint64_t *thr, int lo, int hi, uint64_t dt)
-{
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (thr[mid - 1] <= dt) lo = mid; else hi = mid - 1;
-    }
-    return lo;
-}
-
-// Keys [a, b] intersected with [jh, jh+63], as bits relative to jh.
-__device__ __forceinline__ uint64_t range_bits(int a, int b, int jh)
-{
-    const int lo = max(a, jh) - jh, hi = min(b, jh + HALF - 1) - jh;
-    if (lo > hi) return 0ull;
-    const int n = hi - lo + 1;
-    const uint64_t m = n >= 64 ? ~0ull : ((1ull << n) - 1ull);
-    return m << lo;
-}
-
-// Valid keys of row i among [jh, jh+63] (bit c <-> key jh + c): the contextual prefix for
-// every row; for non-contextual rows the causal (windowed) history keys up to p(i); for a
-// candidate row also itself.  Equivalent to pair_valid over the half tile.
-__device__ __forceinline__ uint64_t row_valid_bits(int i, int jh, const SeqInfo &s, int W)
-{
-    if (i >= s.L) return 0ull;
-    uint64_t m = range_bits(0, s.c - 1, jh);
-    if (i < s.c) return m;
-    const int pi = clamp_pos(i, s.E);
-    const int lo = W > 0 ? max(s.c, pi - W) : s.c;
-    m |= range_bits(lo, min(pi, s.E - 1), jh);
-    if (i >= s.E) m |= range_bits(i, i, jh);
-    return m;
-}
-
-// Fills the time-bucket lookup table; clears *valid when some cell holds two thresholds
-// (bucket thresholds closer than the cell resolution), which disables the table.
-__device__ void build_lut(const uint64_t *thr, int n_thr, LutEntry *lut, int32_t *valid)
-{
-    for (int q = threadIdx.x; q < kLutCells; q += blockDim.x) {
-        const int e = q >> 5, m = q & 31;
-        const uint64_t ylo = (((uint64_t)(32 + m) << e) + 31) >> 5;      // ceil(2^e (32+m)/32)
-        const uint64_t yhi = ((((uint64_t)(33 + m) << e) + 31) >> 5) - 1; // last y in the cell
-        LutEntry ent;
-        ent.next = 0xFFFFFFFFu;
-        ent.base = 0;
-        ent.jump = 0;
-        if (ylo >= 1 && ylo <= yhi) {
-            const uint64_t dlo = ylo - 1, dhi = yhi - 1;
-            const int b = bucket_search(thr, n_thr, dlo);
-            ent.base = (int16_t)b;
-            if (b < n_thr && thr[b] <= dhi) {
-                int n = 1;
-                while (b + n < n_thr && thr[b + n] == thr[b]) ++n;
-                if (b + n < n_thr && thr[b + n] <= dhi) atomicAnd(valid, 0);
-                if (thr[b] > 0xFFFFFFFEull) atomicAnd(valid, 0);
-                ent.next = (uint32_t)min(thr[b], (uint64_t)0xFFFFFFFEull);
-                ent.jump = (int16_t)n;
-            }
-        }
-        lut[q] = ent;
-    }
-}
-
-__device__ __forceinline__ int64_t shfl_xor_i64(int64_t v, int m)
-{
-    return (int64_t)__shfl_xor_sync(0xffffffffu, (long long)v, m);
-}
-
-template <int DQK, int DV>
+// SPLIT: A enters A V as a pair of bf16 values, hi = bf16(A) and lo = bf16(A - hi), so Y
+// carries about 16 significant bits (used when Y is saved for the backward, whose
+// LayerNorm gradient is sensitive to the error of Y).
+template <int DQK, int DV, bool SPLIT>
 __global__ void __launch_bounds__(kTcThreads, 1)
     fwd_tc_kernel(const __grid_constant__ FwdTcArgs args)
 {
@@ -301,10 +215,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 const uint32_t v_addr = sm_base + L::V_OFF + sx * L::VB;
 #pragma unroll
                 for (int kk = 0; kk < BN / 16; ++kk) {
-                    // keys 16kk..16kk+15: half (kk/4) packed at columns [64*half, 64*half+32)
-                    const uint32_t a_tmem = tmem + sx * 128 + (kk >> 2) * 64 + (kk & 3) * 8;
+                    // keys 16kk..16kk+15.  Packed A of half h (keys 64h..64h+63) lives in that
+                    // half's S columns: without SPLIT at [64h, 64h+32); with SPLIT each 32-key
+                    // chunk c holds hi at [64h+32c, +16) and lo at [64h+32c+16, +16)
+                    const uint32_t a_tmem =
+                        SPLIT ? tmem + sx * 128 + (kk >> 2) * 64 + ((kk >> 1) & 1) * 32 + (kk & 1) * 8
+                              : tmem + sx * 128 + (kk >> 2) * 64 + (kk & 3) * 8;
                     const uint64_t bd = sw128_desc(v_addr + kk * 2048, kBlockBytes, 1024);
                     umma_bf16_ts(tmem + kOCol, a_tmem, bd, idesc_pv, (x > 0 || kk > 0) ? 1u : 0u);
+                    if (SPLIT) umma_bf16_ts(tmem + kOCol, a_tmem + 16, bd, idesc_pv, 1u);
                 }
                 umma_commit(&bars[S_FREE + sx]);
                 umma_commit(&bars[KV_EMPTY + sx]);
@@ -537,20 +456,38 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 }
                 // SiLU(x) = x sigmoid(x) = h + h tanh(h), h = x/2; mask after the nonlinearity
                 uint32_t pk[16];
+                float a_full[32];
 #pragma unroll
                 for (int c2 = 0; c2 < 16; ++c2) {
-                    float a2[2];
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
                         const int c = 2 * c2 + e;
-                        const float hx = fmaf(half_alpha, __uint_as_float(ra[c]), 0.5f * av[c]);
-                        const float a = fmaf(hx, tanh_approx(hx), hx);
-                        a2[e] = full ? a : (((vbits >> c) & 1u) ? a : 0.f);
+                        float a;
+                        if (SPLIT) {   // accurate sigmoid for the training forward
+                            const float xs = fmaf(p.alpha, __uint_as_float(ra[c]), av[c]);
+                            a = xs * __fdividef(1.0f, 1.0f + __expf(-xs));
+                        } else {
+                            const float hx = fmaf(half_alpha, __uint_as_float(ra[c]), 0.5f * av[c]);
+                            a = fmaf(hx, tanh_approx(hx), hx);
+                        }
+                        a_full[c] = full ? a : (((vbits >> c) & 1u) ? a : 0.f);
                     }
-                    pk[c2] = pack_bf16x2(a2[0], a2[1]);
+                    pk[c2] = pack_bf16x2(a_full[2 * c2], a_full[2 * c2 + 1]);
                 }
-                // bf16 A over the first 32 of this warpgroup's 64 S columns
-                tmem_st16(tmem + lane_base + st * 128 + wg * HALF + ch * 16, pk);
+                // bf16 A written back over S columns this thread has already read
+                if (SPLIT) {
+                    uint32_t plo[16];
+#pragma unroll
+                    for (int c2 = 0; c2 < 16; ++c2) {
+                        const float h0 = __uint_as_float(pk[c2] << 16);
+                        const float h1 = __uint_as_float(pk[c2] & 0xFFFF0000u);
+                        plo[c2] = pack_bf16x2(a_full[2 * c2] - h0, a_full[2 * c2 + 1] - h1);
+                    }
+                    tmem_st16(tmem + lane_base + st * 128 + wg * HALF + ch * 32, pk);
+                    tmem_st16(tmem + lane_base + st * 128 + wg * HALF + ch * 32 + 16, plo);
+                } else {
+                    tmem_st16(tmem + lane_base + st * 128 + wg * HALF + ch * 16, pk);
+                }
             }
             tmem_wait_st();
             tc_fence_before();
@@ -590,7 +527,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 tmap_encode_fn()
+template <int DQK, int DV>
+cudaError_t launch_tc(const FwdTcArgs &a, bool split, cudaStream_t st)
+{
+    using L = FwdLayout<DQK, DV>;
+    auto kern = split ? fwd_tc_kernel<DQK, DV, true> : fwd_tc_kernel<DQK, DV, false>;
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
+    if (e != cudaSuccess) return e;
+    dim3 grid((a.p.N + BM - 1) / BM, a.p.B, a.p.H);
+    kern<<<grid, kTcThreads, L::ALLOC, st>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+static PFN_cuTensorMapEncodeTiled_v12000 tmap_encode_fn()
 {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
     if (!fn) {
@@ -605,7 +557,7 @@ PFN_cuTensorMapEncodeTiled_v12000 tmap_encode_fn()
 }
 
 // [T, H, d] bf16 row-major as a 3-D tensor (d, H, T); box 64 x 1 x 128, 128-byte swizzle.
-bool encode_tmap(CUtensorMap *m, const void *base, int d, int H, int64_t T)
+bool encode_tmap_bf16(CUtensorMap *m, const void *base, int d, int H, int64_t T)
 {
     auto fn = tmap_encode_fn();
     if (!fn) return false;
@@ -619,40 +571,25 @@ bool encode_tmap(CUtensorMap *m, const void *base, int d, int H, int64_t T)
     return r == CUDA_SUCCESS;
 }
 
-template <int DQK, int DV>
-cudaError_t launch_tc(const FwdTcArgs &a, cudaStream_t st)
-{
-    using L = FwdLayout<DQK, DV>;
-    auto kern = fwd_tc_kernel<DQK, DV>;
-    cudaError_t e =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
-    if (e != cudaSuccess) return e;
-    dim3 grid((a.p.N + BM - 1) / BM, a.p.B, a.p.H);
-    kern<<<grid, kTcThreads, L::ALLOC, st>>>(a);
-    return cudaGetLastError();
-}
-
-}  // namespace
-
 bool tc_fwd_supported(int dqk, int dv, int64_t T)
 {
     return (dqk == 64 || dqk == 128) && (dv == 64 || dv == 128) && T < ((int64_t)1 << 31);
 }
 
 cudaError_t launch_tc_fwd(const DevParams &p, const void *q, const void *k, const void *v,
-                          float *y, cudaStream_t st)
+                          float *y, bool training, cudaStream_t st)
 {
     FwdTcArgs a;
     std::memset(&a, 0, sizeof(a));
     a.p = p;
     a.y = y;
-    if (!encode_tmap(&a.tq, q, p.dqk, p.H, p.T) || !encode_tmap(&a.tk, k, p.dqk, p.H, p.T) ||
-        !encode_tmap(&a.tv, v, p.dv, p.H, p.T))
+    if (!encode_tmap_bf16(&a.tq, q, p.dqk, p.H, p.T) || !encode_tmap_bf16(&a.tk, k, p.dqk, p.H, p.T) ||
+        !encode_tmap_bf16(&a.tv, v, p.dv, p.H, p.T))
         return cudaErrorInvalidValue;
-    if (p.dqk == 128 && p.dv == 128) return launch_tc<128, 128>(a, st);
-    if (p.dqk == 128 && p.dv == 64) return launch_tc<128, 64>(a, st);
-    if (p.dqk == 64 && p.dv == 128) return launch_tc<64, 128>(a, st);
-    if (p.dqk == 64 && p.dv == 64) return launch_tc<64, 64>(a, st);
+    if (p.dqk == 128 && p.dv == 128) return launch_tc<128, 128>(a, training, st);
+    if (p.dqk == 128 && p.dv == 64) return launch_tc<128, 64>(a, training, st);
+    if (p.dqk == 64 && p.dv == 128) return launch_tc<64, 128>(a, training, st);
+    if (p.dqk == 64 && p.dv == 64) return launch_tc<64, 64>(a, training, st);
     return cudaErrorInvalidValue;
 }
 

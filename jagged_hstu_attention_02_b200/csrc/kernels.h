@@ -1,6 +1,7 @@
 // kernels.h -- launchers of the device kernels (host-callable, C++ linkage, internal).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -14,10 +15,12 @@ cudaError_t launch_simt_fwd(const DevParams &p, const void *q, const void *k, co
 template <typename T>
 cudaError_t launch_ln_gate(const DevParams &p, const float *y, const void *u, void *out,
                            float *mean, float *rstd, cudaStream_t st);
+// dy receives fp32 values (dy_bf16 false) or bf16 hi parts at dy and lo parts at dy + T*D
+// (dy_bf16 true).
 template <typename T>
 cudaError_t launch_ln_gate_bwd(const DevParams &p, const void *dout, const void *u,
                                const float *y, const float *mean, const float *rstd, void *du,
-                               float *dy, cudaStream_t st);
+                               void *dy, bool dy_bf16, cudaStream_t st);
 template <typename T>
 cudaError_t launch_simt_bwd(const DevParams &p, const void *q, const void *k, const void *v,
                             const float *dy, float *dq_acc, void *dk, void *dv, float *d_rel,
@@ -25,10 +28,21 @@ cudaError_t launch_simt_bwd(const DevParams &p, const void *q, const void *k, co
 template <typename T>
 cudaError_t launch_convert(const float *src, void *dst, int64_t n, cudaStream_t st);
 
-// tcgen05 forward attention (bf16): Y = (1/N) sum_j A_ij V_j in fp32.
+// tcgen05 forward attention (bf16): Y = (1/N) sum_j A_ij V_j in fp32.  `training` selects
+// the variant whose Y carries ~16 significant bits (A split into bf16 hi + lo parts).
 bool tc_fwd_supported(int dqk, int dv, int64_t T);
 cudaError_t launch_tc_fwd(const DevParams &p, const void *q, const void *k, const void *v,
-                          float *y, cudaStream_t st);
+                          float *y, bool training, cudaStream_t st);
+
+// tcgen05 backward attention (bf16): dQ added into an fp32 accumulator (zeroed by the
+// caller), dK/dV written, table gradients added into d_rel/d_tb (zeroed by the caller).
+bool tc_bwd_supported(int dqk, int dv, int64_t T);
+cudaError_t launch_tc_bwd(const DevParams &p, const void *q, const void *k, const void *v,
+                          const void *dy_bf16 /* hi, then lo at + T*D */, float *dq_acc, void *dk, void *dv, float *d_rel,
+                          float *d_tb, cudaStream_t st);
+
+// [T, H, d] bf16 row-major as a 3-D TMA tensor (d, H, T): box 64 x 1 x 128, 128-byte swizzle.
+bool encode_tmap_bf16(CUtensorMap *m, const void *base, int d, int H, int64_t T);
 
 cudaError_t launch_debug_mask(const DevParams &p, int seq, int seq_len, uint32_t *bits,
                               cudaStream_t st);

@@ -237,12 +237,15 @@ __global__ void __launch_bounds__(kThreads)
 
 // One warp per token: dU = dO (.) Zhat, dZ = dO (.) U,
 // dY = rstd * (dZ - mean(dZ) - Zhat * mean(dZ (.) Zhat)).
-template <typename T>
+// With DYT = bf16, dY is written as a pair of bf16 arrays, hi = bf16(dY) at dy and
+// lo = bf16(dY - hi) at dy + T*D, so that tensor-core products with dY keep about 16
+// significant bits (LayerNorm makes dY orthogonal to Y, and sums over dY can cancel).
+template <typename T, typename DYT>
 __global__ void __launch_bounds__(kThreads)
     ln_gate_bwd_kernel(const __grid_constant__ DevParams p, const T *__restrict__ dout,
                        const T *__restrict__ u, const float *__restrict__ y,
                        const float *__restrict__ mean, const float *__restrict__ rstd,
-                       T *__restrict__ du, float *__restrict__ dy)
+                       T *__restrict__ du, DYT *__restrict__ dy)
 {
     const int lane = threadIdx.x & 31;
     const int64_t row = (int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
@@ -276,7 +279,12 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
     for (int c = 0; c < 64; ++c) {
         const int e = lane + 32 * c;
-        if (e < D) dy[row * D + e] = rs * (dz[c] - m1 - z[c] * m2);
+        if (e < D) {
+            const float g = rs * (dz[c] - m1 - z[c] * m2);
+            const DYT hi = from_f32<DYT>(g);
+            dy[row * D + e] = hi;
+            if (sizeof(DYT) == 2) dy[p.T * D + row * D + e] = from_f32<DYT>(g - to_f32<DYT>(hi));
+        }
     }
 }
 
@@ -499,12 +507,16 @@ cudaError_t launch_ln_gate(const DevParams &p, const float *y, const void *u, vo
 template <typename T>
 cudaError_t launch_ln_gate_bwd(const DevParams &p, const void *dout, const void *u,
                                const float *y, const float *mean, const float *rstd, void *du,
-                               float *dy, cudaStream_t st)
+                               void *dy, bool dy_bf16, cudaStream_t st)
 {
     const int rows_per_block = kThreads / 32;
     const int64_t blocks = (p.T + rows_per_block - 1) / rows_per_block;
-    ln_gate_bwd_kernel<T><<<(unsigned)blocks, kThreads, 0, st>>>(
-        p, (const T *)dout, (const T *)u, y, mean, rstd, (T *)du, dy);
+    if (dy_bf16)
+        ln_gate_bwd_kernel<T, __nv_bfloat16><<<(unsigned)blocks, kThreads, 0, st>>>(
+            p, (const T *)dout, (const T *)u, y, mean, rstd, (T *)du, (__nv_bfloat16 *)dy);
+    else
+        ln_gate_bwd_kernel<T, float><<<(unsigned)blocks, kThreads, 0, st>>>(
+            p, (const T *)dout, (const T *)u, y, mean, rstd, (T *)du, (float *)dy);
     return cudaGetLastError();
 }
 
@@ -545,11 +557,11 @@ template cudaError_t launch_ln_gate<__nv_bfloat16>(const DevParams &, const floa
                                                    cudaStream_t);
 template cudaError_t launch_ln_gate_bwd<float>(const DevParams &, const void *, const void *,
                                                const float *, const float *, const float *,
-                                               void *, float *, cudaStream_t);
+                                               void *, void *, bool, cudaStream_t);
 template cudaError_t launch_ln_gate_bwd<__nv_bfloat16>(const DevParams &, const void *,
                                                        const void *, const float *,
                                                        const float *, const float *, void *,
-                                                       float *, cudaStream_t);
+                                                       void *, bool, cudaStream_t);
 template cudaError_t launch_simt_bwd<float>(const DevParams &, const void *, const void *,
                                             const void *, const float *, float *, void *, void *,
                                             float *, float *, cudaStream_t);
