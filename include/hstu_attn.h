@@ -158,6 +158,33 @@ hstu_status_t hstu_attn_debug_mask(const hstu_attn_params_t *params, const int64
  */
 hstu_status_t hstu_attn_time_thresholds(double div, int32_t nb, uint64_t *out);
 
+/*
+ * Forward for callers that cannot allocate device memory (no counterpart in the paper; it
+ * is a deployment convenience).  Some callers cannot provide the workspace hstu_attn_fwd
+ * asks for: a plugin inside a framework that owns all device memory and offers no
+ * allocation hook, or a latency-critical serving loop in which cudaMalloc, which can
+ * synchronise the device, is not allowed.  This entry point computes the same inference
+ * forward as hstu_attn_fwd (out only; no saved activations) with its scratch in a fixed
+ * 32 MiB array that the library declares in device memory; each GPU that loads the library
+ * keeps that array until the process exits.  It allocates and frees nothing.
+ *   - Arguments: as hstu_attn_fwd, without saved_y/mean/rstd and without a workspace.
+ *   - Limit: the scratch need is 256 + 4 * total_tokens * num_heads * d_v bytes; a request
+ *     above 32 MiB returns HSTU_ERR_WORKSPACE_TOO_SMALL before anything is enqueued.
+ *   - Set-up: the first call on each device looks up the array's device address (with that
+ *     device current); make that first call before any stream capture.
+ *   - Sharing: all calls on a device share the one array, which keeps the last call's
+ *     contents (the status word is cleared by every call).  Calls that overlap on the GPU
+ *     (other streams, other threads) race on it: serialise them.
+ *   - Device-data errors skip the offending sequences as in hstu_attn_fwd, but their status
+ *     bits stay inside the shared scratch; callers that need them use hstu_attn_fwd.
+ */
+hstu_status_t hstu_attn_fwd_noalloc(const hstu_attn_params_t *params, const void *q,
+                                    const void *k, const void *v, const void *u,
+                                    const int64_t *seq_offsets, const int32_t *num_contextuals,
+                                    const int32_t *num_targets, const int64_t *timestamps,
+                                    const float *rel_bias, const float *time_bias, void *out,
+                                    void *stream);
+
 /* Kernel stages of fwd/bwd, for hstu_attn_set_stage_events. */
 #define HSTU_STAGE_FWD_ATTN 0   /* forward attention (scores, bias, SiLU, mask, A V) */
 #define HSTU_STAGE_FWD_NORM 1   /* forward LayerNorm + U gating */
