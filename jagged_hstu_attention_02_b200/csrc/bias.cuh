@@ -131,10 +131,17 @@ struct HalfTime {
     int32_t cmpA, cmpB, t_rel;
 };
 
+// Exact bucket of dt < 2^31 - 1 through the lookup table.
+__device__ __forceinline__ int lut_bucket(const LutEntry *lut, uint32_t dt)
+{
+    const LutEntry e = lut[lut_cell(dt)];
+    return e.base + (dt >= e.next ? e.jump : 0);
+}
+
 __device__ __forceinline__ HalfTime half_time_setup(const uint64_t *thr, int n_thr,
                                                     const float *tbs, int NB, bool row_in,
                                                     int64_t t_row, int64_t hmin, int64_t hmax,
-                                                    bool h32, bool lut_ok)
+                                                    bool h32, bool lut_ok, const LutEntry *lut)
 {
     HalfTime h;
     h.my_mode = 0;
@@ -157,8 +164,13 @@ __device__ __forceinline__ HalfTime half_time_setup(const uint64_t *thr, int n_t
             const uint64_t c = (uint64_t)hmax - (uint64_t)t_row;
             dhi = a > c ? a : c;
         }
-        h.blo = bucket_in(thr, 0, n_thr, dlo);
-        bhi = bucket_in(thr, h.blo, n_thr, dhi);
+        if (lut_ok && dhi < (uint64_t)(INT32_MAX - 1)) {
+            h.blo = lut_bucket(lut, (uint32_t)dlo);
+            bhi = lut_bucket(lut, (uint32_t)dhi);
+        } else {
+            h.blo = bucket_in(thr, 0, n_thr, dlo);
+            bhi = bucket_in(thr, h.blo, n_thr, dhi);
+        }
         const bool fits = h32 && dhi < (uint64_t)(INT32_MAX - 1);
         if (fits) h.t_rel = (int32_t)((uint64_t)t_row - (uint64_t)hmin);
         if (bhi == h.blo) {

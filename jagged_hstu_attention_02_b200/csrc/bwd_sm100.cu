@@ -375,7 +375,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             int tmode = 0;
             if (use_ts) {
                 ht = half_time_setup(thr, p.n_thr, tbs, p.NB, key_in, tsj, meta->tmin[wg],
-                                     meta->tmax[wg], meta->ok32[wg] != 0, lut_ok);
+                                     meta->tmax[wg], meta->ok32[wg] != 0, lut_ok, lut);
                 tmode = __reduce_max_sync(0xffffffffu, ht.my_mode);
             }
             float tsum_lo = 0.f, tsum_hi = 0.f;    // dS sums per bucket in modes 0/1

@@ -15,15 +15,16 @@
 // Persistent: one CTA per SM walks the units in longest-first order (query tiles from the
 // last to the first, so the tiles with the most keys start first), so the per-CTA set-up
 // (barriers, TMEM, bias tables, bucket lookup table) happens once per SM and the loads of
-// the next unit overlap the tail of the current one.  Warp roles (12 warps): warp 0 lane 0
-// loads Q and K (3 K stages), warp 2 lane 0 loads V (2 stages; warp 2 also owns TMEM),
-// warp 1 lane 0 issues the MMAs, warp 3 stages each key tile's timestamps and their range,
-// warps 4-7 and 8-11 are two epilogue warpgroups, each owning 64 of the 128 key columns of
-// every query row (thread = row = TMEM lane).  TMEM: S double-buffered [0,256), output
-// accumulator double-buffered across units [256,384) and [384,512).
+// the next unit (Q is double-buffered) overlap the tail of the current one.  Warp roles (20
+// warps): warp 0 lane 0 loads Q and K, warp 2 lane 0 loads V (warp 2 also owns TMEM), warp
+// 1 lane 0 issues the MMAs, warp 3 stages each key tile's timestamps and per-quarter
+// ranges, warps 4-19 are four epilogue warpgroups, each owning 32 of the 128 key columns
+// of every query row (thread = row = TMEM lane).  TMEM: S double-buffered [0,256), A in
+// its own columns [256,384) so S is released as soon as the epilogue has read it, output
+// accumulator [384,512).
 //
-// Bias evaluation per (row, 64-key half tile):  the time bucket is computed once for the
-// smallest and largest |dt| the half can produce (from the half's timestamp range); when
+// Bias evaluation per (row, 32-key quarter tile):  the time bucket is computed once for
+// the smallest and largest |dt| the quarter can produce (from its timestamp range); when
 // both agree (the common case away from the diagonal) the time bias is a per-row constant.
 // The rel index runs p(i)-j down a contiguous window of the table when no clamping occurs.
 // Mask evaluation is skipped on tiles the mask covers fully.  Every wait is bounded; a
@@ -42,22 +43,25 @@ using namespace sm100;
 
 namespace {
 
-constexpr int BM = 128, BN = 128, HALF = kHalf;
-constexpr int kTcThreads = 384;
+constexpr int BM = 128, BN = 128, QW = 32;   // QW: key columns per epilogue warpgroup
+constexpr int kEpiWarps = 16;                  // four warpgroups
+constexpr int kTcThreads = 128 + 32 * kEpiWarps;
 constexpr int kRelSmemMax = 4096;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kBlockBytes = 128 * 128;   // one 128-row x 64-element bf16 swizzle block
-constexpr uint32_t kOCol = 256;          // TMEM column of output accumulator 0 (1 at +128)
-constexpr int KST = 3, VST = 2;          // K and V stages
+constexpr uint32_t kPCol = 256;          // TMEM columns of A (packed bf16)
+constexpr uint32_t kOCol = 384;          // TMEM columns of the output accumulator
+constexpr int KST = 2, VST = 2, QST = 2; // K, V and Q stages
+// mean relative loss of cutting an fp32 to bf16 (dropping 16 bits), ~0.72 * 2^-8
+constexpr float kTruncBump = 1.0028f;
 
-enum Bar { Q_FULL = 0, Q_EMPTY = 1, K_FULL = 2, K_EMPTY = 5, V_FULL = 8, V_EMPTY = 10,
-           S_FULL = 12, S_FREE = 14, P_FULL = 16, META_FULL = 18, O_FULL = 20, O_FREE = 22,
-           MMA_DONE = 24, NUM_BARS = 25 };
+enum Bar { Q_FULL = 0, Q_EMPTY = 2, K_FULL = 4, K_EMPTY = 6, V_FULL = 8, V_EMPTY = 10,
+           S_FULL = 12, S_FREE = 14, P_FULL = 16, P_FREE = 18, META_FULL = 20, EPI_DONE = 22,
+           O_FULL = 24, O_FREE = 25, MMA_DONE = 26, NUM_BARS = 27 };
 
 struct TileMeta {
-    int64_t tmin[2], tmax[2];   // timestamp range of each 64-key half (valid keys only)
-    int32_t ok32[2];            // the half's range is below 2^31 - 1: 32-bit relative stamps valid
-    int32_t pad[2];
+    int64_t tmin[4], tmax[4];   // timestamp range of each 32-key quarter (valid keys only)
+    int32_t ok32[4];            // the quarter's range is below 2^31 - 1: 32-bit stamps valid
 };
 
 template <int DQK, int DV>
@@ -66,7 +70,7 @@ struct FwdLayout {
     static constexpr int KB = BN * DQK * 2;
     static constexpr int VB = BN * DV * 2;
     static constexpr int Q_OFF = 0;
-    static constexpr int K_OFF = Q_OFF + QB;
+    static constexpr int K_OFF = Q_OFF + QST * QB;
     static constexpr int V_OFF = K_OFF + KST * KB;
     static constexpr int BAR_OFF = V_OFF + VST * VB;
     static constexpr int SLOT_OFF = BAR_OFF + 8 * 32;
@@ -140,14 +144,24 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity)
     return __all_sync(0xffffffffu, mbar_wait(bar, parity));
 }
 
+// One arrival per warp on `bar` (counted per warp), after the whole warp got here.
+__device__ __forceinline__ void warp_arrive(uint64_t *bar)
+{
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+}
+
 // SPLIT: A enters A V as a pair of bf16 values, hi = bf16(A) and lo = bf16(A - hi), so Y
 // carries about 16 significant bits (used when Y is saved for the backward, whose
-// LayerNorm gradient is sensitive to the error of Y).
+// LayerNorm gradient is sensitive to the error of Y).  Without SPLIT, A has two TMEM
+// buffers of 64 columns; with SPLIT one buffer of 128 (per 32-key quarter w: hi at
+// 32w..32w+15, lo at 32w+16..32w+31).
 template <int DQK, int DV, bool SPLIT>
 __global__ void __launch_bounds__(kTcThreads, 1)
     fwd_tc_kernel(const __grid_constant__ FwdTcArgs args)
 {
     using L = FwdLayout<DQK, DV>;
+    constexpr int NP = SPLIT ? 1 : 2;   // A buffers
     const DevParams &p = args.p;
 
     extern __shared__ uint8_t smem_raw[];
@@ -161,26 +175,32 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     int32_t *tsk32 = reinterpret_cast<int32_t *>(sm + L::TSK32_OFF);
     LutEntry *lutp = reinterpret_cast<LutEntry *>(sm + L::LUT_OFF);
     uint64_t *thr = reinterpret_cast<uint64_t *>(sm + L::THR_OFF);
-    float *tbh = reinterpret_cast<float *>(sm + L::TB_OFF);    // 0.5 * time table
-    float *relh = reinterpret_cast<float *>(sm + L::REL_OFF);  // 0.5 * rel table
+    float *tbh = reinterpret_cast<float *>(sm + L::TB_OFF);    // scaled half time table
+    float *relh = reinterpret_cast<float *>(sm + L::REL_OFF);  // scaled half rel table
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
     if (threadIdx.x == 0) {
         for (int x = 0; x < NUM_BARS; ++x) mbar_init(&bars[x], 1);
         for (int x = 0; x < 2; ++x) {
-            mbar_init(&bars[P_FULL + x], 256);
+            mbar_init(&bars[S_FREE + x], kEpiWarps);
+            mbar_init(&bars[P_FULL + x], kEpiWarps);
             mbar_init(&bars[META_FULL + x], 32);
-            mbar_init(&bars[O_FREE + x], 256);
+            mbar_init(&bars[EPI_DONE + x], kEpiWarps);
         }
+        mbar_init(&bars[O_FREE], kEpiWarps);
         fence_mbar_init();
         *lut_valid = 1;
     }
     if (warp == 2) tmem_alloc(slot, kTmemCols);
+    // Tables hold half the bias.  The inference variant also scales by kTruncBump: its h is
+    // cut to bf16 by dropping the low 16 bits, and the bump removes the mean bias of that
+    // truncation (remaining error within one bf16 ulp).
+    const float tscale = SPLIT ? 0.5f : 0.5f * kTruncBump;
     for (int x = threadIdx.x; x < p.n_thr; x += kTcThreads) thr[x] = p.thr[x];
-    for (int x = threadIdx.x; x < p.NB; x += kTcThreads) tbh[x] = 0.5f * p.tb[x];
+    for (int x = threadIdx.x; x < p.NB; x += kTcThreads) tbh[x] = tscale * p.tb[x];
     const bool rel_in_smem = p.R <= kRelSmemMax;
     if (rel_in_smem)
-        for (int x = threadIdx.x; x < p.R; x += kTcThreads) relh[x] = 0.5f * p.rel[x];
+        for (int x = threadIdx.x; x < p.R; x += kTcThreads) relh[x] = tscale * p.rel[x];
     __syncthreads();
     if (p.NB > 0) build_lut(thr, p.n_thr, lutp, lut_valid);
     tc_fence_before();
@@ -198,12 +218,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             int n = 0, g = 0;
             bool ok = true;
             while (ok && un.next()) {
-                const int i0 = un.qt * BM, row0 = (int)un.s.start;
-                if (n >= 1 && !mbar_wait(&bars[Q_EMPTY], (n - 1) & 1)) { ok = false; break; }
-                mbar_arrive_expect_tx(&bars[Q_FULL], L::QB);
+                const int i0 = un.qt * BM, row0 = (int)un.s.start, qs = n % QST;
+                if (n >= QST && !mbar_wait(&bars[Q_EMPTY + qs], (n / QST - 1) & 1)) {
+                    ok = false;
+                    break;
+                }
+                mbar_arrive_expect_tx(&bars[Q_FULL + qs], L::QB);
                 for (int kb = 0; kb < DQK / 64; ++kb)
-                    tma_load_3d(sm + L::Q_OFF + kb * kBlockBytes, &args.tq, &bars[Q_FULL],
-                                kb * 64, un.h, row0 + i0);
+                    tma_load_3d(sm + L::Q_OFF + qs * L::QB + kb * kBlockBytes, &args.tq,
+                                &bars[Q_FULL + qs], kb * 64, un.h, row0 + i0);
                 TileIter t(un.s, i0, p.W);
                 while (t.next()) {
                     const int st = g % KST;
@@ -222,7 +245,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             if (!ok) report_timeout(p);
             // loads issued must land before the CTA exits (bounded)
             bool drained = true;
-            if (n >= 1) drained &= mbar_wait(&bars[Q_FULL], (n - 1) & 1);
+            for (int x = n - 1; x >= 0 && x >= n - QST; --x)
+                drained &= mbar_wait(&bars[Q_FULL + x % QST], (x / QST) & 1);
             for (int x = g - 1; x >= 0 && x >= g - KST; --x)
                 drained &= mbar_wait(&bars[K_FULL + x % KST], (x / KST) & 1);
             if (!drained) report_timeout(p);
@@ -256,48 +280,47 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 drained &= mbar_wait(&bars[V_FULL + x % VST], (x / VST) & 1);
             if (!drained) report_timeout(p);
         }
-    } else if (warp == 1) {
+    }
+    else if (warp == 1) {
         if (lane == 0) {
             // ---------------------------------------------------------------- MMA issuer
             constexpr uint32_t idesc_qk = idesc_bf16(BM, BN, false, false);
             constexpr uint32_t idesc_pv = idesc_bf16(BM, DV, false, true);
-            const uint32_t q_addr = sm_base + L::Q_OFF;
-            // A V for tile g of unit n (O buffer n&1); first/last tile of the unit
+            const uint32_t o_tmem = tmem + kOCol;
+            // A V for tile g of unit n; first/last tile of the unit
             auto issue_pv = [&](int g, int n, bool first, bool last) -> bool {
-                const int sx = g & 1, ob = n & 1;
-                if (!mbar_wait(&bars[P_FULL + sx], (g >> 1) & 1)) return false;
+                const int ps = g % NP;
+                if (!mbar_wait(&bars[P_FULL + ps], (g / NP) & 1)) return false;
                 if (!mbar_wait(&bars[V_FULL + g % VST], (g / VST) & 1)) return false;
-                if (first && n >= 2 && !mbar_wait(&bars[O_FREE + ob], ((n >> 1) - 1) & 1))
-                    return false;
+                if (first && n >= 1 && !mbar_wait(&bars[O_FREE], (n - 1) & 1)) return false;
                 tc_fence_after();
                 const uint32_t v_addr = sm_base + L::V_OFF + (g % VST) * L::VB;
-                const uint32_t o_tmem = tmem + kOCol + ob * 128;
 #pragma unroll
                 for (int kk = 0; kk < BN / 16; ++kk) {
-                    // keys 16kk..16kk+15.  Packed A of half h (keys 64h..64h+63) lives in that
-                    // half's S columns: without SPLIT at [64h, 64h+32); with SPLIT each 32-key
-                    // chunk c holds hi at [64h+32c, +16) and lo at [64h+32c+16, +16)
+                    // keys 16kk..16kk+15; see the layout of A above
                     const uint32_t a_tmem =
-                        SPLIT ? tmem + sx * 128 + (kk >> 2) * 64 + ((kk >> 1) & 1) * 32 + (kk & 1) * 8
-                              : tmem + sx * 128 + (kk >> 2) * 64 + (kk & 3) * 8;
+                        SPLIT ? tmem + kPCol + (kk >> 1) * 32 + (kk & 1) * 8
+                              : tmem + kPCol + ps * 64 + kk * 8;
                     const uint64_t bd = sw128_desc(v_addr + kk * 2048, kBlockBytes, 1024);
                     umma_bf16_ts(o_tmem, a_tmem, bd, idesc_pv, (!first || kk > 0) ? 1u : 0u);
                     if (SPLIT) umma_bf16_ts(o_tmem, a_tmem + 16, bd, idesc_pv, 1u);
                 }
-                umma_commit(&bars[S_FREE + sx]);
+                umma_commit(&bars[P_FREE + ps]);
                 umma_commit(&bars[V_EMPTY + g % VST]);
-                if (last) umma_commit(&bars[O_FULL + ob]);
+                if (last) umma_commit(&bars[O_FULL]);
                 return true;
             };
             UnitIter un(p, args.nqt, false);
             int n = 0, g = 0;
             bool ok = true;
-            bool pend = false;                  // a PV waiting for its A
+            bool pend = false;                  // an A V waiting for its A
             int pg = 0, pn = 0;
             bool pfirst = false;
             while (ok && un.next()) {
-                if (!mbar_wait(&bars[Q_FULL], n & 1)) { ok = false; break; }
+                const int qs = n % QST;
+                if (!mbar_wait(&bars[Q_FULL + qs], (n / QST) & 1)) { ok = false; break; }
                 tc_fence_after();
+                const uint32_t q_addr = sm_base + L::Q_OFF + qs * L::QB;
                 TileIter t(un.s, un.qt * BM, p.W);
                 bool first = true, more = t.next();
                 while (more) {
@@ -320,7 +343,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     umma_commit(&bars[S_FULL + st]);
                     umma_commit(&bars[K_EMPTY + ks]);
                     more = t.next();
-                    if (!more) umma_commit(&bars[Q_EMPTY]);   // Q free once its last QK^T ends
+                    if (!more) umma_commit(&bars[Q_EMPTY + qs]);   // Q free after its last QK^T
                     // the previous tile's A V (possibly of the previous unit, which it closes)
                     if (pend && !issue_pv(pg, pn, pfirst, pn != n)) { ok = false; break; }
                     pend = true;
@@ -338,8 +361,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             umma_commit(&bars[MMA_DONE]);
             if (!mbar_wait(&bars[MMA_DONE], 0)) report_timeout(p);
         }
-    }
-    else if (warp == 3) {
+    } else if (warp == 3) {
         // -------------------------------------------------------------------- tile metadata
         const bool use_ts = p.NB > 0;
         UnitIter un(p, args.nqt, false);
@@ -350,53 +372,49 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             TileIter t(s, un.qt * BM, p.W);
             while (t.next()) {
                 const int st = g & 1;
-                if (g >= 2 && !warp_wait(&bars[S_FREE + st], ((g >> 1) - 1) & 1)) {
+                // the epilogue is done with this stage's stamps (tile g - 2)
+                if (g >= 2 && !warp_wait(&bars[EPI_DONE + st], ((g >> 1) - 1) & 1)) {
                     report_timeout(p);
                     ok = false;
                     break;
                 }
                 if (use_ts) {
                     const int j0 = t.kt * BN;
-                    int64_t v[4];
-                    int64_t mn[2] = {INT64_MAX, INT64_MAX}, mx[2] = {INT64_MIN, INT64_MIN};
+                    int64_t v[4], mn[4], mx[4];
 #pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
+                    for (int q4 = 0; q4 < 4; ++q4) {      // key lane + 32 q4 lies in quarter q4
                         const int j = j0 + lane + 32 * q4;
                         v[q4] = 0;
+                        mn[q4] = INT64_MAX;
+                        mx[q4] = INT64_MIN;
                         if (j < s.L) {
                             v[q4] = p.ts[s.start + clamp_pos(j, s.E)];
-                            mn[q4 >> 1] = min(mn[q4 >> 1], v[q4]);
-                            mx[q4 >> 1] = max(mx[q4 >> 1], v[q4]);
+                            mn[q4] = mx[q4] = v[q4];
                         }
                     }
 #pragma unroll
-                    for (int hh = 0; hh < 2; ++hh)
+                    for (int q4 = 0; q4 < 4; ++q4)
 #pragma unroll
                         for (int o = 16; o > 0; o >>= 1) {
-                            mn[hh] = min(mn[hh], shfl_xor_i64(mn[hh], o));
-                            mx[hh] = max(mx[hh], shfl_xor_i64(mx[hh], o));
+                            mn[q4] = min(mn[q4], shfl_xor_i64(mn[q4], o));
+                            mx[q4] = max(mx[q4], shfl_xor_i64(mx[q4], o));
                         }
-                    int ok32[2];
-#pragma unroll
-                    for (int hh = 0; hh < 2; ++hh)
-                        ok32[hh] = mn[hh] > mx[hh] ||
-                                   (uint64_t)mx[hh] - (uint64_t)mn[hh] < (uint64_t)INT32_MAX;
 #pragma unroll
                     for (int q4 = 0; q4 < 4; ++q4) {
-                        const int c = lane + 32 * q4, hh = q4 >> 1;
+                        const int c = lane + 32 * q4;
+                        const bool ok32 = mn[q4] > mx[q4] ||
+                                          (uint64_t)mx[q4] - (uint64_t)mn[q4] < (uint64_t)INT32_MAX;
                         tsk[st * BN + c] = v[q4];
-                        // stamps relative to the half's minimum (0 for keys past the sequence)
-                        tsk32[st * BN + c] = (j0 + c < s.L && ok32[hh])
-                                                 ? (int32_t)((uint64_t)v[q4] - (uint64_t)mn[hh])
+                        // stamps relative to the quarter's minimum (0 for keys past the sequence)
+                        tsk32[st * BN + c] = (j0 + c < s.L && ok32)
+                                                 ? (int32_t)((uint64_t)v[q4] - (uint64_t)mn[q4])
                                                  : 0;
-                    }
-                    if (lane == 0)
-#pragma unroll
-                        for (int hh = 0; hh < 2; ++hh) {
-                            meta[st].tmin[hh] = mn[hh];
-                            meta[st].tmax[hh] = mx[hh];
-                            meta[st].ok32[hh] = ok32[hh];
+                        if (lane == 0) {
+                            meta[st].tmin[q4] = mn[q4];
+                            meta[st].tmax[q4] = mx[q4];
+                            meta[st].ok32[q4] = ok32;
                         }
+                    }
                 }
                 __syncwarp();
                 mbar_arrive(&bars[META_FULL + st]);
@@ -406,14 +424,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     else if (warp >= 4) {
         // -------------------------------------------------------------------- epilogue
-        const int wg = (warp - 4) >> 2;               // 0: keys 0..63, 1: keys 64..127
+        const int wq = (warp - 4) >> 2;               // key quarter: columns [32 wq, 32 wq + 32)
         const int r = (warp & 3) * 32 + lane;         // query row in the tile == TMEM lane
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
         const bool use_ts = p.NB > 0;
         const bool use_rel = p.R > 0;
         const float *relp = rel_in_smem ? relh : p.rel;
-        const float rel_sc = rel_in_smem ? 1.0f : 0.5f;   // relp * rel_sc = half the rel bias
-        const float half_alpha = 0.5f * p.alpha;
+        const float rel_sc = rel_in_smem ? 1.0f : tscale;  // relp * rel_sc = scaled half rel bias
+        const float half_alpha = SPLIT ? 0.5f * p.alpha : 0.5f * kTruncBump * p.alpha;
         const bool lut_ok = *lut_valid != 0;
         UnitIter un(p, args.nqt, false);
         int n = 0, g = 0;
@@ -427,75 +445,77 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const int64_t tsi = (use_ts && row_in) ? p.ts[s.start + pi] : 0;
             TileIter t(s, i0, p.W);
             while (t.next()) {
-                const int st = g & 1;
-                const int jh = t.kt * BN + wg * HALF;     // first key of this warpgroup's half
-                const bool full = tile_all_valid(i0, i0 + BM - 1, jh, jh + HALF - 1, s, p.W);
+                const int st = g & 1, ps = g % NP;
+                const int jq = t.kt * BN + wq * QW;      // first key of this warpgroup's quarter
+                const bool full = tile_all_valid(i0, i0 + BM - 1, jq, jq + QW - 1, s, p.W);
                 if (!warp_wait(&bars[META_FULL + st], (g >> 1) & 1) ||
                     !warp_wait(&bars[S_FULL + st], (g >> 1) & 1)) {
                     ok = false;
                     break;
                 }
+                tc_fence_after();
+                uint32_t ra[32];
+                tmem_ld32(tmem + lane_base + st * 128 + wq * QW, ra);
+                tmem_wait_ld();
+                reg_fence(ra);
+                tc_fence_before();
+                warp_arrive(&bars[S_FREE + st]);      // S is in registers: release it
 
-                // ---- per (row, half tile) structure; path choices are made warp-uniform
-                const uint64_t vmask = full ? ~0ull : row_valid_bits(i, jh, s, p.W);
-                const int rbase = pi - jh;            // rel index of key jh + c is rbase - c
-                const bool rdirect = __all_sync(0xffffffffu, !use_rel || (rbase - (HALF - 1) >= 0 &&
-                                                                            rbase <= p.R - 1));
-                // time bias (halved): mode 0 per-row constant, 1 one bucket boundary, 2 lookup
-                // table, 3 64-bit search
+                // ---- per (row, quarter tile) structure; path choices are made warp-uniform
+                const uint32_t vmask = full ? 0xFFFFFFFFu : (uint32_t)row_valid_bits(i, jq, s, p.W);
+                const int rbase = pi - jq;            // rel index of key jq + c is rbase - c
+                const bool rdirect =
+                    __all_sync(0xffffffffu, !use_rel || (rbase - (QW - 1) >= 0 && rbase <= p.R - 1));
                 HalfTime ht = {};
                 int tmode = 0;
                 if (use_ts) {
-                    ht = half_time_setup(thr, p.n_thr, tbh, p.NB, row_in, tsi, meta[st].tmin[wg],
-                                         meta[st].tmax[wg], meta[st].ok32[wg] != 0, lut_ok);
+                    ht = half_time_setup(thr, p.n_thr, tbh, p.NB, row_in, tsi, meta[st].tmin[wq],
+                                         meta[st].tmax[wq], meta[st].ok32[wq] != 0, lut_ok, lutp);
                     tmode = __reduce_max_sync(0xffffffffu, ht.my_mode);
                 }
-                const int32_t *tk32 = tsk32 + st * BN + wg * HALF;
-                const int64_t *tk64 = tsk + st * BN + wg * HALF;
-
+                const int32_t *tk32 = tsk32 + st * BN + wq * QW;
+                const int64_t *tk64 = tsk + st * BN + wq * QW;
+                // A's buffer is free once the A V of tile g - NP has completed
+                if (g >= NP && !warp_wait(&bars[P_FREE + ps], ((g / NP) - 1) & 1)) {
+                    ok = false;
+                    break;
+                }
                 tc_fence_after();
-#pragma unroll 1
-                for (int ch = 0; ch < 2; ++ch) {
-                    const uint32_t s_col = tmem + lane_base + st * 128 + wg * HALF + ch * 32;
-                    uint32_t ra[32];
-                    tmem_ld32(s_col, ra);
-                    tmem_wait_ld();
-                    reg_fence(ra);
-                    const uint32_t vbits = (uint32_t)(vmask >> (32 * ch));
-                    const int cb = ch * 32;
-                    float bh[32];   // half of the bias, time part first
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    const int cb = hf * 16;
+                    float bh[16];   // scaled half of the bias, time part first
                     if (tmode == 0) {
 #pragma unroll
-                        for (int c = 0; c < 32; ++c) bh[c] = ht.tb_lo;
+                        for (int c = 0; c < 16; ++c) bh[c] = ht.tb_lo;
                     } else if (tmode == 1) {
 #pragma unroll
-                        for (int c = 0; c < 32; ++c) {
+                        for (int c = 0; c < 16; ++c) {
                             const int32_t tj = tk32[cb + c];
                             bh[c] = (tj <= ht.cmpA || tj >= ht.cmpB) ? ht.tb_hi : ht.tb_lo;
                         }
                     } else if (tmode == 2) {
 #pragma unroll
-                        for (int c = 0; c < 32; ++c) {
+                        for (int c = 0; c < 16; ++c) {
                             int32_t d = ht.t_rel - tk32[cb + c];
                             uint32_t dt = (uint32_t)(d < 0 ? -d : d);
                             dt = min(dt, (uint32_t)INT32_MAX - 1u);
-                            const LutEntry e = lutp[lut_cell(dt)];
-                            const float v = tbh[e.base + (dt >= e.next ? e.jump : 0)];
+                            const float v = tbh[lut_bucket(lutp, dt)];
                             bh[c] = ht.lane_const ? ht.tb_lo : v;
                         }
                     } else {
 #pragma unroll
-                        for (int c = 0; c < 32; ++c)
+                        for (int c = 0; c < 16; ++c)
                             bh[c] = tbh[bucket_search(thr, p.n_thr, abs_diff_u64(tsi, tk64[cb + c]))];
                     }
                     if (use_rel) {
                         if (rdirect) {
                             const float *rr = relp + (rbase - cb);
 #pragma unroll
-                            for (int c = 0; c < 32; ++c) bh[c] = fmaf(rr[-c], rel_sc, bh[c]);
+                            for (int c = 0; c < 16; ++c) bh[c] = fmaf(rr[-c], rel_sc, bh[c]);
                         } else {
 #pragma unroll
-                            for (int c = 0; c < 32; ++c) {
+                            for (int c = 0; c < 16; ++c) {
                                 int ri = rbase - cb - c;
                                 ri = ri < 0 ? 0 : (ri > p.R - 1 ? p.R - 1 : ri);
                                 bh[c] = fmaf(relp[ri], rel_sc, bh[c]);
@@ -503,69 +523,79 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         }
                     }
                     // SiLU(x) = x sigmoid(x) = h + h tanh(h), h = x/2; mask after the nonlinearity
-                    uint32_t pk[16];
-                    float a_full[32];
+                    uint32_t pk[8];
+                    const uint32_t vb = vmask >> cb;
+                    if constexpr (SPLIT) {
+                        // training forward: accurate sigmoid in fp32, A split into hi + lo
+                        uint32_t plo[8];
 #pragma unroll
-                    for (int c2 = 0; c2 < 16; ++c2) {
+                        for (int c2 = 0; c2 < 8; ++c2) {
+                            float a[2];
 #pragma unroll
-                        for (int e = 0; e < 2; ++e) {
-                            const int c = 2 * c2 + e;
-                            float a;
-                            if (SPLIT) {   // accurate sigmoid for the training forward
-                                const float xs = fmaf(p.alpha, __uint_as_float(ra[c]), 2.0f * bh[c]);
-                                a = xs * __fdividef(1.0f, 1.0f + __expf(-xs));
-                            } else {
-                                const float hx = fmaf(half_alpha, __uint_as_float(ra[c]), bh[c]);
-                                a = fmaf(hx, tanh_approx(hx), hx);
+                            for (int e = 0; e < 2; ++e) {
+                                const int c = 2 * c2 + e;
+                                const float xs = fmaf(p.alpha, __uint_as_float(ra[cb + c]), 2.0f * bh[c]);
+                                const float v = xs * __fdividef(1.0f, 1.0f + __expf(-xs));
+                                a[e] = full ? v : (((vb >> c) & 1u) ? v : 0.f);
                             }
-                            a_full[c] = full ? a : (((vbits >> c) & 1u) ? a : 0.f);
+                            pk[c2] = pack_bf16x2(a[0], a[1]);
+                            plo[c2] = pack_bf16x2(a[0] - __uint_as_float(pk[c2] << 16),
+                                                  a[1] - __uint_as_float(pk[c2] & 0xFFFF0000u));
                         }
-                        pk[c2] = pack_bf16x2(a_full[2 * c2], a_full[2 * c2 + 1]);
-                    }
-                    // bf16 A written back over S columns this thread has already read
-                    if (SPLIT) {
-                        uint32_t plo[16];
-#pragma unroll
-                        for (int c2 = 0; c2 < 16; ++c2) {
-                            const float h0 = __uint_as_float(pk[c2] << 16);
-                            const float h1 = __uint_as_float(pk[c2] & 0xFFFF0000u);
-                            plo[c2] = pack_bf16x2(a_full[2 * c2] - h0, a_full[2 * c2 + 1] - h1);
-                        }
-                        tmem_st16(tmem + lane_base + st * 128 + wg * HALF + ch * 32, pk);
-                        tmem_st16(tmem + lane_base + st * 128 + wg * HALF + ch * 32 + 16, plo);
+                        tmem_st8(tmem + lane_base + kPCol + wq * 32 + hf * 8, pk);
+                        tmem_st8(tmem + lane_base + kPCol + wq * 32 + 16 + hf * 8, plo);
                     } else {
-                        tmem_st16(tmem + lane_base + st * 128 + wg * HALF + ch * 16, pk);
+                        // inference forward: h in fp32, then tanh and h + h tanh(h) on bf16 pairs
+                        // (A is rounded to bf16 for the tensor core either way)
+#pragma unroll
+                        for (int c2 = 0; c2 < 8; ++c2) {
+                            const float x0 = fmaf(half_alpha, __uint_as_float(ra[cb + 2 * c2]), bh[2 * c2]);
+                            const float x1 =
+                                fmaf(half_alpha, __uint_as_float(ra[cb + 2 * c2 + 1]), bh[2 * c2 + 1]);
+                            // bf16 pair = the high halves of x0, x1 (one byte permute)
+                            const uint32_t h2 =
+                                __byte_perm(__float_as_uint(x0), __float_as_uint(x1), 0x7632);
+                            uint32_t a2 = fma_bf16x2(h2, tanh_bf16x2(h2), h2);
+                            if (!full)
+                                a2 &= (((vb >> (2 * c2)) & 1u) ? 0x0000FFFFu : 0u) |
+                                      (((vb >> (2 * c2 + 1)) & 1u) ? 0xFFFF0000u : 0u);
+                            pk[c2] = a2;
+                        }
+                        tmem_st8(tmem + lane_base + kPCol + ps * 64 + wq * 16 + hf * 8, pk);
                     }
                 }
                 tmem_wait_st();
                 tc_fence_before();
-                mbar_arrive(&bars[P_FULL + st]);
+                warp_arrive(&bars[P_FULL + ps]);
+                warp_arrive(&bars[EPI_DONE + st]);    // stamps and ranges of this stage read
                 ++g;
             }
             if (!ok) break;
-            // ---- the unit's output: Y = (1/N) O, this warpgroup's half of the columns
-            const int ob = n & 1;
-            if (!warp_wait(&bars[O_FULL + ob], (n >> 1) & 1)) { ok = false; break; }
+            // ---- the unit's output: Y = (1/N) O; this warpgroup's quarter of the columns
+            if (!warp_wait(&bars[O_FULL], n & 1)) { ok = false; break; }
             tc_fence_after();
-            float *yr = args.y + (s.start + i) * (int64_t)p.D + un.h * DV;
-#pragma unroll 1
-            for (int c = wg * (DV / 64); c < (wg + 1) * (DV / 64); ++c) {
-                uint32_t ra[32];
-                tmem_ld32(tmem + lane_base + kOCol + ob * 128 + c * 32, ra);
-                tmem_wait_ld();
-                reg_fence(ra);
-                if (row_in) {
-                    float4 *dst = reinterpret_cast<float4 *>(yr + c * 32);
-#pragma unroll
-                    for (int x = 0; x < 8; ++x)
-                        dst[x] = make_float4(__uint_as_float(ra[4 * x]) * p.inv_N,
-                                             __uint_as_float(ra[4 * x + 1]) * p.inv_N,
-                                             __uint_as_float(ra[4 * x + 2]) * p.inv_N,
-                                             __uint_as_float(ra[4 * x + 3]) * p.inv_N);
-                }
+            constexpr int OC = DV / 4;                // 32 or 16 output columns per warpgroup
+            float *yr = args.y + (s.start + i) * (int64_t)p.D + un.h * DV + wq * OC;
+            uint32_t ro[32];
+            if (OC == 32) {
+                tmem_ld32(tmem + lane_base + kOCol + wq * OC, ro);
+            } else {
+                uint32_t (&r16)[16] = *reinterpret_cast<uint32_t(*)[16]>(ro);
+                tmem_ld16(tmem + lane_base + kOCol + wq * OC, r16);
             }
+            tmem_wait_ld();
+            reg_fence(ro);
             tc_fence_before();
-            mbar_arrive(&bars[O_FREE + ob]);
+            warp_arrive(&bars[O_FREE]);
+            if (row_in) {
+                float4 *dst = reinterpret_cast<float4 *>(yr);
+#pragma unroll
+                for (int x = 0; x < OC / 4; ++x)
+                    dst[x] = make_float4(__uint_as_float(ro[4 * x]) * p.inv_N,
+                                         __uint_as_float(ro[4 * x + 1]) * p.inv_N,
+                                         __uint_as_float(ro[4 * x + 2]) * p.inv_N,
+                                         __uint_as_float(ro[4 * x + 3]) * p.inv_N);
+            }
             ++n;
         }
         if (!ok) report_timeout(p);
@@ -579,6 +609,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tmem_dealloc(tmem, kTmemCols);
     }
 }
+
 
 int num_sms()
 {
