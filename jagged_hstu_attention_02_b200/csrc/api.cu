@@ -127,8 +127,10 @@ size_t bwd_ws_bytes(const hstu_attn_params_t *p)
 {
     size_t n = kHeaderBytes;
     n += align_up((size_t)p->total_tokens * p->num_heads * p->d_v * 4, 256);     // dY
-    if (p->dtype != HSTU_F32)
+    if (p->dtype != HSTU_F32) {
         n += align_up((size_t)p->total_tokens * p->num_heads * p->d_qk * 4, 256);  // dQ fp32
+        n += (size_t)kBwdMaxCtas * kMaxTimeBuckets * 4;   // per-CTA time-gradient rows
+    }
     return n;
 }
 
@@ -300,6 +302,8 @@ hstu_status_t hstu_attn_bwd(const hstu_attn_params_t *p, const void *dout, const
     const bool f32 = p->dtype == HSTU_F32;
     const bool tc = !f32 && tc_bwd_supported(p->d_qk, p->d_v, p->total_tokens);
     float *dq_acc = f32 ? reinterpret_cast<float *>(dq) : reinterpret_cast<float *>(ws);
+    float *tb_slots = f32 ? nullptr
+                          : reinterpret_cast<float *>(ws + align_up((size_t)nq * 4, 256));
     HSTU_CUDA_TRY(cudaMemsetAsync(dq_acc, 0, sizeof(float) * nq, s));
     {
         StageScope scope(HSTU_STAGE_BWD_NORM, s);
@@ -317,7 +321,7 @@ hstu_status_t hstu_attn_bwd(const hstu_attn_params_t *p, const void *dout, const
                                                  d_time_bias, s));
         } else if (tc) {
             HSTU_CUDA_TRY(launch_tc_bwd(d, q, k, v, dy, dq_acc, dk, dv, d_rel_bias, d_time_bias,
-                                        s));
+                                        tb_slots, s));
             HSTU_CUDA_TRY(launch_convert<__nv_bfloat16>(dq_acc, dq, nq, s));
         } else {
             HSTU_CUDA_TRY(launch_simt_bwd<__nv_bfloat16>(d, q, k, v, dy, dq_acc, dk, dv,

@@ -9,16 +9,27 @@
 // "Similar shape, different aggregation"; the mask multiplies after the nonlinearity, so
 // masked pairs get exactly zero gradient ("Do not copy softmax masking mechanically").
 //
-// One CTA per (128-key tile, sequence, head); it walks the 128-row query tiles that see
-// the keys.  Thread = key row = TMEM lane, so scores are computed transposed:
+// Persistent CTAs walk work units (128-key tile, sequence, head), units with the most query
+// tiles first; a unit walks the 128-row query tiles that see its keys.  Thread = key row =
+// TMEM lane, so scores are computed transposed:
 //   S^T = K Q^T and dP^T = V dY^T          (tcgen05, bf16 in smem, fp32 in TMEM)
-//   epilogue: A^T (bf16, over S^T in TMEM) and dS^T (bf16, 128B-swizzled in smem)
+//   epilogue: A^T (bf16, over S^T in TMEM) and dS^T (bf16, 128B-swizzled in smem, in the
+//             buffer of the dY low parts, which dP^T has finished with)
 //   dV += A^T dY (A from TMEM), dK += dS^T Q, dQ_tile = dS K (dS^T read as an MN-major A)
-// dV and dK accumulate in TMEM across query tiles; each dQ tile is added to an fp32
-// accumulator in global memory with vector atomics.  Table gradients go through
-// shared-memory histograms.  Warp roles as in the forward: TMA producer, MMA issuer, TMEM
-// owner, query-timestamp staging, and two epilogue warpgroups that split the query
-// columns.  Every wait is bounded.
+// dV and dK accumulate in TMEM across the query tiles of a unit; each dQ tile is added to an
+// fp32 accumulator in global memory with vector reductions.
+//
+// Table gradients never take a shared-memory atomic per pair (a float atomic add on shared
+// memory retries under contention, and the pairs of one query hit few buckets):
+//   rel: within a 32-key x 32-query block the index is the diagonal i - j, so each warp sums
+//        the diagonals in registers by shifting partial sums one lane per column, and adds
+//        the 63 diagonal sums with two scatters; pairs whose index is clamped (candidate
+//        rows, far or bidirectional pairs) go to per-lane sums with one index each.
+//   time: along a key row the bucket changes rarely (timestamps ascend with position), so
+//        each lane sums runs of equal buckets and adds a run with one fire-and-forget global
+//        reduction into a histogram private to the CTA, folded into the output at the end.
+// Warp roles: TMA producer, MMA issuer, TMEM owner, query-timestamp staging, and four
+// epilogue warpgroups that split the query columns.  Every wait is bounded.
 #include <cudaTypedefs.h>
 
 #include <cstring>
@@ -33,21 +44,27 @@ using namespace sm100;
 
 namespace {
 
-constexpr int BM = 128, BN = 128, HALF = kHalf;
-constexpr int kThreads = 384;
+constexpr int BM = 128, BN = 128;
+constexpr int QW = 32;                  // query columns per epilogue warpgroup
+constexpr int kEpiWarps = 16;
+constexpr int kThreads = 128 + 32 * kEpiWarps;
 constexpr int kRelSmemMax = 2048;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kBlockBytes = 128 * 128;
 // TMEM columns: S^T -> A^T [0,128); dP^T -> dQ tile [128,256); dV [256,384); dK [384,512)
 constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 384;
 
-enum Bar { KV_FULL = 0, QD_FULL = 1, QD_EMPTY = 2, SD_FULL = 3, META_FULL = 4, P_FULL = 5,
-           DQ_FULL = 6, DQ_FREE = 7, ACC_FULL = 8, MMA_DONE = 9, NUM_BARS = 10 };
+enum Bar {
+    KV_FULL = 0, KV_EMPTY = 1, QD_FULL = 2, QD_EMPTY = 3, SD_FULL = 4, META_FULL = 5,  // +2
+    EPI_DONE = 7,                                                                     // +2
+    P_FULL = 9, DQ_FULL = 10, DQ_FREE = 11, ACC_FULL = 12, ACC_FREE = 13, MMA_DONE = 14,
+    NUM_BARS = 15
+};
 
+// Time-stamp ranges of the four 32-query quarters of a query tile.
 struct QMeta {
-    int64_t tmin[2], tmax[2];
-    int32_t ok32[2];
-    int32_t pad[2];
+    int64_t tmin[4], tmax[4];
+    int32_t ok32[4];
 };
 
 template <int DQK, int DV>
@@ -56,26 +73,27 @@ struct BwdLayout {
     static constexpr int VB = BN * DV * 2;
     static constexpr int QB = BM * DQK * 2;
     static constexpr int YB = BM * DV * 2;
-    static constexpr int SB = BN * BM * 2;
+    static constexpr int SB = BN * BM * 2;        // dS^T, bf16
+    static constexpr int LB = YB > SB ? YB : SB;  // dY low parts, then dS^T
     static constexpr int K_OFF = 0;
     static constexpr int V_OFF = K_OFF + KB;
     static constexpr int Q_OFF = V_OFF + VB;
     static constexpr int Y_OFF = Q_OFF + QB;
-    static constexpr int YL_OFF = Y_OFF + YB;
-    static constexpr int DS_OFF = YL_OFF + YB;
-    static constexpr int BAR_OFF = DS_OFF + SB;
+    static constexpr int YL_OFF = Y_OFF + YB;     // also DS
+    static constexpr int BAR_OFF = YL_OFF + LB;
     static constexpr int SLOT_OFF = BAR_OFF + 8 * 16;
     static constexpr int META_OFF = SLOT_OFF + 16;
-    static constexpr int TSQ_OFF = META_OFF + (int)sizeof(QMeta);
-    static constexpr int TSQ32_OFF = TSQ_OFF + BM * 8;
-    static constexpr int LUT_OFF = TSQ32_OFF + BM * 4;
+    static constexpr int TSQ_OFF = META_OFF + 2 * (int)sizeof(QMeta);
+    static constexpr int TSQ32_OFF = TSQ_OFF + 2 * BM * 8;
+    static constexpr int LUT_OFF = TSQ32_OFF + 2 * BM * 4;
     static constexpr int THR_OFF = LUT_OFF + kLutCells * 8;
     static constexpr int TB_OFF = THR_OFF + 8 * kMaxTimeBuckets;
-    static constexpr int HTB_OFF = TB_OFF + 4 * kMaxTimeBuckets;
-    static constexpr int REL_OFF = HTB_OFF + 4 * kMaxTimeBuckets;
+    static constexpr int REL_OFF = TB_OFF + 4 * kMaxTimeBuckets;
     static constexpr int HREL_OFF = REL_OFF + 4 * kRelSmemMax;
     static constexpr int TOTAL = HREL_OFF + 4 * kRelSmemMax;
     static constexpr int ALLOC = TOTAL + 1024;
+    static_assert(NUM_BARS <= 16, "barrier area");
+    static_assert(TSQ_OFF % 8 == 0 && LUT_OFF % 8 == 0, "alignment");
 };
 
 struct BwdTcArgs {
@@ -84,6 +102,35 @@ struct BwdTcArgs {
     float *dq_acc;                 // [T, H, d_qk] fp32, zeroed by the caller
     __nv_bfloat16 *dk, *dv;        // [T, H, d]
     float *d_rel, *d_tb;
+    float *tb_slots;               // [gridDim.x, kMaxTimeBuckets] scratch, one row per CTA
+    int nkt;                       // key tiles of the longest admissible sequence
+};
+
+// Work units (key tile kt, sequence b, head h), key tile 0 first: a unit over key tile kt
+// visits the query tiles kt .. of its sequence, so low kt carries the most work.
+struct UnitIter {
+    const DevParams &p;
+    int nkt;
+    int64_t u, total;
+    bool report;
+    SeqInfo s;
+    int kt, b, h;
+    __device__ UnitIter(const DevParams &p_, int nkt_, bool report_)
+        : p(p_), nkt(nkt_), u((int64_t)blockIdx.x - gridDim.x),
+          total((int64_t)nkt_ * p_.B * p_.H), report(report_) {}
+    __device__ bool next()
+    {
+        while ((u += gridDim.x) < total) {
+            const int64_t bh = (int64_t)p.B * p.H;
+            kt = (int)(u / bh);
+            const int rem = (int)(u % bh);
+            b = rem / p.H;
+            h = rem % p.H;
+            s = load_seq(p, b, report && kt == 0 && h == 0);
+            if (kt * BN < s.L) return true;
+        }
+        return false;
+    }
 };
 
 // The query tiles [i0, i0+BM) that see key tile [j0, j0+BN), in order.
@@ -110,11 +157,237 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity)
     return __all_sync(0xffffffffu, mbar_wait(bar, parity));
 }
 
+// One arrival per warp on `bar` (counted per warp), after the whole warp got here.
+__device__ __forceinline__ void warp_arrive(uint64_t *bar)
+{
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+}
+
 __device__ __forceinline__ void red_add_v4(float *addr, float a, float b, float c, float d)
 {
     asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
                  "f"(c), "f"(d)
                  : "memory");
+}
+
+__device__ __forceinline__ void red_add(float *addr, float a)
+{
+    asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(a) : "memory");
+}
+
+__device__ __forceinline__ float ld_cg(const float *addr)
+{
+    float v;
+    asm volatile("ld.global.cg.f32 %0, [%1];" : "=f"(v) : "l"(addr) : "memory");
+    return v;
+}
+
+// Adds v to the rel-bias gradient at index ri (shared histogram or the global output).
+__device__ __forceinline__ void rel_add(float *hrel, float *d_rel, bool in_smem, int ri, float v)
+{
+    if (in_smem) atomicAdd(hrel + ri, v);
+    else red_add(d_rel + ri, v);
+}
+
+// Per-lane state of one epilogue thread (key row j of the unit) across the query tiles.
+struct KeyLane {
+    int j, pj;
+    bool key_in;
+    int64_t tsj;
+    // rel gradient: shifted diagonal sums (A: diagonals 31 - lane, B: -1 - lane of the
+    // 32 x 32 block) and the clamped pairs (candidate rows, index p(E-1) - p(j); negative
+    // distance, index 0; beyond the table, index R-1)
+    float sysA, sysB, cand, negs, fars;
+    // time gradient: the open run of equal buckets
+    int cur_b;
+    float run;
+};
+
+// One 32-key x 32-query block of the epilogue: reads S^T and dP^T of the block from TMEM,
+// writes A^T (bf16 pairs, over the block's own S^T columns) and dS^T (bf16, swizzled smem),
+// and accumulates the table gradients into the lane state.  TM is the warp-uniform time
+// mode of half_time_setup (0 when there is no time bias).
+struct EpiBlock {
+    uint32_t t_s, t_dp, t_a;      // TMEM addresses of the block's S^T, dP^T and A^T columns
+    uint32_t ds_row;              // smem address of this key's dS^T row (first 16-byte chunk)
+    int ds_chunk0, rsw;           // first chunk of the block in the row, swizzle (row & 7)
+    int iq;                       // first query of the block
+    int rbase;                    // p(iq) - p(j) when rdirect
+    int Em1;                      // p(i) = min(i, Em1)
+    bool full, rdirect, use_rel, use_ts, rel_in_smem;
+    uint32_t vbits;               // valid queries of this key (bit c <-> query iq + c)
+    const int32_t *tq32;          // the block's query stamps relative to the quarter minimum
+    const int64_t *tq64;          // and absolute
+    const float *relp;
+    const uint64_t *thr;
+    const float *tbs;
+    const LutEntry *lut;
+    float *tb_slot;
+};
+
+template <int TM>
+__device__ __forceinline__ void epi_block(const DevParams &p, const EpiBlock &e,
+                                          const HalfTime &ht, KeyLane &k, float &t_lo,
+                                          float &t_hi)
+{
+    const int lane = threadIdx.x & 31;
+    if (TM == 0 && e.use_ts && k.key_in) {
+        if (ht.blo != k.cur_b) {
+            if (k.run != 0.f) red_add(e.tb_slot + k.cur_b, k.run);
+            k.cur_b = ht.blo;
+            k.run = 0.f;
+        }
+    }
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+        uint32_t rs[16], rd[16];
+        tmem_ld16(e.t_s + hf * 16, rs);
+        tmem_ld16(e.t_dp + hf * 16, rd);
+        tmem_wait_ld();
+        reg_fence(rs);
+        reg_fence(rd);
+        uint32_t pa[8], pd[8];
+#pragma unroll
+        for (int c2 = 0; c2 < 8; ++c2) {
+            float av[2], dv2[2];
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                const int c = 2 * c2 + q, cc = hf * 16 + c;
+                const int i = e.iq + cc;
+                const bool valid = e.full || ((e.vbits >> cc) & 1u);
+                // ---- bias
+                float bias = 0.f;
+                int bk = 0;
+                if (TM == 0) {
+                    bias = ht.tb_lo;
+                } else if (TM == 1) {
+                    const int32_t t = e.tq32[cc];
+                    const bool hi = t <= ht.cmpA || t >= ht.cmpB;
+                    bias = hi ? ht.tb_hi : ht.tb_lo;
+                    bk = hi ? 1 : 0;
+                } else if (TM == 2) {
+                    if (ht.lane_const) {
+                        bias = ht.tb_lo;
+                        bk = ht.blo;
+                    } else {
+                        const int32_t d = ht.t_rel - e.tq32[cc];
+                        uint32_t dt = (uint32_t)(d < 0 ? -d : d);
+                        dt = min(dt, (uint32_t)INT32_MAX - 1u);
+                        bk = lut_bucket(e.lut, dt);
+                        bias = e.tbs[bk];
+                    }
+                } else {
+                    bk = bucket_search(e.thr, p.n_thr, abs_diff_u64(k.tsj, e.tq64[cc]));
+                    bias = e.tbs[bk];
+                }
+                int rraw = 0, ri = 0;
+                if (e.use_rel) {
+                    if (e.rdirect) {
+                        ri = e.rbase + cc;
+                    } else {
+                        rraw = min(i, e.Em1) - k.pj;
+                        ri = rraw < 0 ? 0 : (rraw > p.R - 1 ? p.R - 1 : rraw);
+                    }
+                    bias += e.relp[ri];
+                }
+                // ---- s = alpha q.k + b; SiLU(s) = s sigma(s); SiLU'(s) = sigma (1 + s (1 - sigma)).
+                // sigma from the accurate exponential: table gradients sum dS over many pairs
+                // and can cancel, so dS needs close to fp32 accuracy
+                const float xs = fmaf(p.alpha, __uint_as_float(rs[c]), bias);
+                const float sig = __fdividef(1.0f, 1.0f + __expf(-xs));
+                const float silu = xs * sig;
+                const float dsilu = sig * fmaf(xs, 1.0f - sig, 1.0f);
+                const float a = valid ? silu * p.inv_N : 0.f;
+                const float ds = valid ? __uint_as_float(rd[c]) * dsilu * p.inv_N : 0.f;
+                av[q] = a;
+                dv2[q] = ds;
+                // ---- rel gradient: shift the diagonal sums one lane down, add this column
+                if (e.use_rel) {
+                    float vd = ds;
+                    if (!e.rdirect) {
+                        if (i > e.Em1) {              // candidate row (warp-uniform)
+                            k.cand += ds;
+                            vd = 0.f;
+                        } else if (rraw != ri) {
+                            if (rraw < 0) k.negs += ds; else k.fars += ds;
+                            vd = 0.f;
+                        }
+                    }
+                    const float ain = __shfl_sync(0xffffffffu, k.sysA, (lane + 31) & 31);
+                    const float bin = __shfl_sync(0xffffffffu, k.sysB, (lane + 31) & 31);
+                    k.sysB = lane == 0 ? ain : bin;
+                    k.sysA = (lane == 0 ? 0.f : ain) + vd;
+                }
+                // ---- time gradient
+                if (e.use_ts) {
+                    if (TM == 0) {
+                        k.run += ds;
+                    } else if (TM == 1) {
+                        if (bk) t_hi += ds; else t_lo += ds;
+                    } else if (valid) {
+                        if (bk != k.cur_b) {
+                            if (k.run != 0.f) red_add(e.tb_slot + k.cur_b, k.run);
+                            k.cur_b = bk;
+                            k.run = 0.f;
+                        }
+                        k.run += ds;
+                    }
+                }
+            }
+            pa[c2] = pack_bf16x2(av[0], av[1]);
+            pd[c2] = pack_bf16x2(dv2[0], dv2[1]);
+        }
+        tmem_st8(e.t_a + hf * 8, pa);
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            const int chunk = e.ds_chunk0 + hf * 2 + q;
+            st_shared_v4(e.ds_row + ((chunk ^ e.rsw) << 4), pd[4 * q], pd[4 * q + 1],
+                         pd[4 * q + 2], pd[4 * q + 3]);
+        }
+    }
+}
+
+// Adds the rel-gradient sums of a finished block and resets them.  Diagonal d (relative to
+// the block) has index iq - jw + d, jw = the warp's first key.
+__device__ __forceinline__ void flush_rel(const DevParams &p, KeyLane &k, int iq, int jw,
+                                          int Em1, float *hrel, float *d_rel, bool in_smem)
+{
+    const int lane = threadIdx.x & 31;
+    const int base = iq - jw;
+    const int ra = base + 31 - lane, rb = base - 1 - lane;
+    if (k.sysA != 0.f && ra >= 0 && ra < p.R) rel_add(hrel, d_rel, in_smem, ra, k.sysA);
+    if (k.sysB != 0.f && rb >= 0 && rb < p.R) rel_add(hrel, d_rel, in_smem, rb, k.sysB);
+    if (k.cand != 0.f) {
+        int rc = Em1 - k.pj;
+        rc = rc < 0 ? 0 : (rc > p.R - 1 ? p.R - 1 : rc);
+        rel_add(hrel, d_rel, in_smem, rc, k.cand);
+    }
+    if (__any_sync(0xffffffffu, k.negs != 0.f || k.fars != 0.f)) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            k.negs += __shfl_xor_sync(0xffffffffu, k.negs, o);
+            k.fars += __shfl_xor_sync(0xffffffffu, k.fars, o);
+        }
+        if (lane == 0) {
+            if (k.negs != 0.f) rel_add(hrel, d_rel, in_smem, 0, k.negs);
+            if (k.fars != 0.f) rel_add(hrel, d_rel, in_smem, p.R - 1, k.fars);
+        }
+    }
+    k.sysA = k.sysB = k.cand = k.negs = k.fars = 0.f;
+}
+
+// Adds v to the time-gradient run state for bucket b (closing the open run if it differs).
+__device__ __forceinline__ void run_add(KeyLane &k, float *slot, int b, float v)
+{
+    if (v == 0.f) return;
+    if (b != k.cur_b) {
+        if (k.run != 0.f) red_add(slot + k.cur_b, k.run);
+        k.cur_b = b;
+        k.run = v;
+    } else {
+        k.run += v;
+    }
 }
 
 template <int DQK, int DV>
@@ -123,11 +396,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 {
     using L = BwdLayout<DQK, DV>;
     const DevParams &p = args.p;
-    const int kt = blockIdx.x, b = blockIdx.y, h = blockIdx.z;
-    const SeqInfo s = load_seq(p, b, kt == 0 && h == 0 && threadIdx.x == 0);
-    const int j0 = kt * BN;
-    if (j0 >= s.L) return;
-
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
@@ -140,16 +408,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     LutEntry *lut = reinterpret_cast<LutEntry *>(sm + L::LUT_OFF);
     uint64_t *thr = reinterpret_cast<uint64_t *>(sm + L::THR_OFF);
     float *tbs = reinterpret_cast<float *>(sm + L::TB_OFF);
-    float *htb = reinterpret_cast<float *>(sm + L::HTB_OFF);
     float *rels = reinterpret_cast<float *>(sm + L::REL_OFF);
     float *hrel = reinterpret_cast<float *>(sm + L::HREL_OFF);
+    float *tb_slot = args.tb_slots + (size_t)blockIdx.x * kMaxTimeBuckets;
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
     if (threadIdx.x == 0) {
         for (int x = 0; x < NUM_BARS; ++x) mbar_init(&bars[x], 1);
-        mbar_init(&bars[META_FULL], 32);
-        mbar_init(&bars[P_FULL], 256);
-        mbar_init(&bars[DQ_FREE], 256);
+        mbar_init(&bars[EPI_DONE], kEpiWarps);
+        mbar_init(&bars[EPI_DONE + 1], kEpiWarps);
+        mbar_init(&bars[P_FULL], kEpiWarps);
+        mbar_init(&bars[DQ_FREE], kEpiWarps);
+        mbar_init(&bars[ACC_FREE], kEpiWarps);
         fence_mbar_init();
         *lut_valid = 1;
     }
@@ -157,7 +427,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int x = threadIdx.x; x < p.n_thr; x += kThreads) thr[x] = p.thr[x];
     for (int x = threadIdx.x; x < p.NB; x += kThreads) {
         tbs[x] = p.tb[x];
-        htb[x] = 0.f;
+        tb_slot[x] = 0.f;
     }
     const bool rel_in_smem = p.R <= kRelSmemMax;
     if (rel_in_smem)
@@ -165,6 +435,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             rels[x] = p.rel[x];
             hrel[x] = 0.f;
         }
+    __threadfence();   // the zeroed slot row is in place before any reduction into it
     __syncthreads();
     if (p.NB > 0) build_lut(thr, p.n_thr, lut, lut_valid);
     tc_fence_before();
@@ -172,7 +443,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem = *slot;
     const uint32_t sm_base = smem_u32(sm);
-    const int row0 = (int)s.start;
 
     if (warp == 0) {
         if (lane == 0) {
@@ -182,34 +452,42 @@ __global__ void __launch_bounds__(kThreads, 1)
             prefetch_tmap(&args.tv);
             prefetch_tmap(&args.tdy);
             prefetch_tmap(&args.tdyl);
-            mbar_arrive_expect_tx(&bars[KV_FULL], L::KB + L::VB);
-            for (int kb = 0; kb < DQK / 64; ++kb)
-                tma_load_3d(sm + L::K_OFF + kb * kBlockBytes, &args.tk, &bars[KV_FULL], kb * 64, h,
-                            row0 + j0);
-            for (int kb = 0; kb < DV / 64; ++kb)
-                tma_load_3d(sm + L::V_OFF + kb * kBlockBytes, &args.tv, &bars[KV_FULL], kb * 64, h,
-                            row0 + j0);
-            QTileIter t(s, j0, p.W);
-            int x = 0;
+            UnitIter un(p, args.nkt, true);
+            int n = 0, g = 0;
             bool ok = true;
-            while (t.next()) {
-                if (x >= 1 && !mbar_wait(&bars[QD_EMPTY], (x - 1) & 1)) { ok = false; break; }
-                const int i0 = t.qt * BM;
-                mbar_arrive_expect_tx(&bars[QD_FULL], L::QB + 2 * L::YB);
+            while (ok && un.next()) {
+                const int row0 = (int)un.s.start, j0 = un.kt * BN;
+                if (n >= 1 && !mbar_wait(&bars[KV_EMPTY], (n - 1) & 1)) { ok = false; break; }
+                mbar_arrive_expect_tx(&bars[KV_FULL], L::KB + L::VB);
                 for (int kb = 0; kb < DQK / 64; ++kb)
-                    tma_load_3d(sm + L::Q_OFF + kb * kBlockBytes, &args.tq, &bars[QD_FULL], kb * 64,
-                                h, row0 + i0);
-                for (int kb = 0; kb < DV / 64; ++kb) {
-                    tma_load_3d(sm + L::Y_OFF + kb * kBlockBytes, &args.tdy, &bars[QD_FULL],
-                                kb * 64, h, row0 + i0);
-                    tma_load_3d(sm + L::YL_OFF + kb * kBlockBytes, &args.tdyl, &bars[QD_FULL],
-                                kb * 64, h, row0 + i0);
+                    tma_load_3d(sm + L::K_OFF + kb * kBlockBytes, &args.tk, &bars[KV_FULL],
+                                kb * 64, un.h, row0 + j0);
+                for (int kb = 0; kb < DV / 64; ++kb)
+                    tma_load_3d(sm + L::V_OFF + kb * kBlockBytes, &args.tv, &bars[KV_FULL],
+                                kb * 64, un.h, row0 + j0);
+                ++n;
+                QTileIter t(un.s, j0, p.W);
+                while (t.next()) {
+                    if (g >= 1 && !mbar_wait(&bars[QD_EMPTY], (g - 1) & 1)) { ok = false; break; }
+                    const int i0 = t.qt * BM;
+                    mbar_arrive_expect_tx(&bars[QD_FULL], L::QB + 2 * L::YB);
+                    for (int kb = 0; kb < DQK / 64; ++kb)
+                        tma_load_3d(sm + L::Q_OFF + kb * kBlockBytes, &args.tq, &bars[QD_FULL],
+                                    kb * 64, un.h, row0 + i0);
+                    for (int kb = 0; kb < DV / 64; ++kb) {
+                        tma_load_3d(sm + L::Y_OFF + kb * kBlockBytes, &args.tdy, &bars[QD_FULL],
+                                    kb * 64, un.h, row0 + i0);
+                        tma_load_3d(sm + L::YL_OFF + kb * kBlockBytes, &args.tdyl, &bars[QD_FULL],
+                                    kb * 64, un.h, row0 + i0);
+                    }
+                    ++g;
                 }
-                ++x;
             }
             if (!ok) report_timeout(p);
-            bool drained = mbar_wait(&bars[KV_FULL], 0);
-            if (x >= 1) drained &= mbar_wait(&bars[QD_FULL], (x - 1) & 1);
+            // every copy has landed before the CTA may exit
+            bool drained = true;
+            if (n >= 1) drained &= mbar_wait(&bars[KV_FULL], (n - 1) & 1);
+            if (g >= 1) drained &= mbar_wait(&bars[QD_FULL], (g - 1) & 1);
             if (!drained) report_timeout(p);
         }
     } else if (warp == 1) {
@@ -221,66 +499,79 @@ __global__ void __launch_bounds__(kThreads, 1)
             constexpr uint32_t id_dq = idesc_bf16(BM, DQK, true, true);      // dS K
             const uint32_t k_addr = sm_base + L::K_OFF, v_addr = sm_base + L::V_OFF;
             const uint32_t q_addr = sm_base + L::Q_OFF, y_addr = sm_base + L::Y_OFF;
-            const uint32_t yl_addr = sm_base + L::YL_OFF;
-            const uint32_t ds_addr = sm_base + L::DS_OFF;
-            bool ok = mbar_wait(&bars[KV_FULL], 0);
-            QTileIter t(s, j0, p.W);
-            int x = 0;
-            while (ok && t.next()) {
-                if (!mbar_wait(&bars[QD_FULL], x & 1)) { ok = false; break; }
-                // the previous tile's dQ readout is done, so every MMA of it completed and
-                // TMEM [0,256) and the dS^T buffer are free
-                if (x >= 1 && !mbar_wait(&bars[DQ_FREE], (x - 1) & 1)) { ok = false; break; }
-                tc_fence_after();
+            const uint32_t yl_addr = sm_base + L::YL_OFF, ds_addr = sm_base + L::YL_OFF;
+            UnitIter un(p, args.nkt, false);
+            int n = 0, g = 0;
+            bool ok = true;
+            while (ok && un.next()) {
+                if (!mbar_wait(&bars[KV_FULL], n & 1)) { ok = false; break; }
+                QTileIter t(un.s, un.kt * BN, p.W);
+                int x = 0;
+                while (t.next()) {
+                    if (!mbar_wait(&bars[QD_FULL], g & 1)) { ok = false; break; }
+                    // the previous tile's dQ has been read: every MMA of it completed, so the
+                    // S^T/A^T and dP^T/dQ columns are free
+                    if (g >= 1 && !mbar_wait(&bars[DQ_FREE], (g - 1) & 1)) { ok = false; break; }
+                    tc_fence_after();
 #pragma unroll
-                for (int kb = 0; kb < DQK / 64; ++kb)
+                    for (int kb = 0; kb < DQK / 64; ++kb)
 #pragma unroll
-                    for (int ks = 0; ks < 4; ++ks) {
-                        const uint64_t a = sw128_desc(k_addr + kb * kBlockBytes + ks * 32, 16, 1024);
-                        const uint64_t bd = sw128_desc(q_addr + kb * kBlockBytes + ks * 32, 16, 1024);
-                        umma_bf16_ss(tmem + kColS, a, bd, id_s, (kb | ks) ? 1u : 0u);
+                        for (int ks = 0; ks < 4; ++ks) {
+                            const uint64_t a = sw128_desc(k_addr + kb * kBlockBytes + ks * 32, 16, 1024);
+                            const uint64_t bd = sw128_desc(q_addr + kb * kBlockBytes + ks * 32, 16, 1024);
+                            umma_bf16_ss(tmem + kColS, a, bd, id_s, (kb | ks) ? 1u : 0u);
+                        }
+                    // dP^T = V (dY_hi + dY_lo)^T
+#pragma unroll
+                    for (int kb = 0; kb < DV / 64; ++kb)
+#pragma unroll
+                        for (int ks = 0; ks < 4; ++ks) {
+                            const uint64_t a = sw128_desc(v_addr + kb * kBlockBytes + ks * 32, 16, 1024);
+                            const uint64_t bd = sw128_desc(y_addr + kb * kBlockBytes + ks * 32, 16, 1024);
+                            const uint64_t bl = sw128_desc(yl_addr + kb * kBlockBytes + ks * 32, 16, 1024);
+                            umma_bf16_ss(tmem + kColDP, a, bd, id_s, (kb | ks) ? 1u : 0u);
+                            umma_bf16_ss(tmem + kColDP, a, bl, id_s, 1u);
+                        }
+                    umma_commit(&bars[SD_FULL]);
+                    if (!mbar_wait(&bars[P_FULL], g & 1)) { ok = false; break; }
+                    // dV and dK of the previous unit have been read out
+                    if (x == 0 && n >= 1 && !mbar_wait(&bars[ACC_FREE], (n - 1) & 1)) {
+                        ok = false;
+                        break;
                     }
-                // dP^T = V (dY_hi + dY_lo)^T
+                    tc_fence_after();
 #pragma unroll
-                for (int kb = 0; kb < DV / 64; ++kb)
-#pragma unroll
-                    for (int ks = 0; ks < 4; ++ks) {
-                        const uint64_t a = sw128_desc(v_addr + kb * kBlockBytes + ks * 32, 16, 1024);
-                        const uint64_t bd = sw128_desc(y_addr + kb * kBlockBytes + ks * 32, 16, 1024);
-                        const uint64_t bl = sw128_desc(yl_addr + kb * kBlockBytes + ks * 32, 16, 1024);
-                        umma_bf16_ss(tmem + kColDP, a, bd, id_s, (kb | ks) ? 1u : 0u);
-                        umma_bf16_ss(tmem + kColDP, a, bl, id_s, 1u);
+                    for (int kk = 0; kk < BM / 16; ++kk) {
+                        // dV += A^T dY: queries 16kk.. packed at columns 32(kk/2) + 8(kk%2)
+                        const uint32_t a_tmem = tmem + kColS + (kk >> 1) * 32 + (kk & 1) * 8;
+                        const uint64_t bd = sw128_desc(y_addr + kk * 2048, kBlockBytes, 1024);
+                        umma_bf16_ts(tmem + kColDV, a_tmem, bd, id_dv, (x > 0 || kk > 0) ? 1u : 0u);
                     }
-                umma_commit(&bars[SD_FULL]);
-                if (!mbar_wait(&bars[P_FULL], x & 1)) { ok = false; break; }
-                tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < BM / 16; ++kk) {
-                    // dV += A^T dY: A^T packed in TMEM (queries 64h.. at columns 64h..64h+31)
-                    const uint32_t a_tmem = tmem + kColS + (kk >> 2) * 64 + (kk & 3) * 8;
-                    const uint64_t bd = sw128_desc(y_addr + kk * 2048, kBlockBytes, 1024);
-                    umma_bf16_ts(tmem + kColDV, a_tmem, bd, id_dv, (x > 0 || kk > 0) ? 1u : 0u);
-                }
+                    for (int kk = 0; kk < BM / 16; ++kk) {
+                        // dK += dS^T Q: dS^T K-major [keys x queries], Q as MN-major B
+                        const uint64_t a = sw128_desc(ds_addr + (kk >> 2) * kBlockBytes + (kk & 3) * 32,
+                                                      16, 1024);
+                        const uint64_t bd = sw128_desc(q_addr + kk * 2048, kBlockBytes, 1024);
+                        umma_bf16_ss(tmem + kColDK, a, bd, id_dk, (x > 0 || kk > 0) ? 1u : 0u);
+                    }
 #pragma unroll
-                for (int kk = 0; kk < BM / 16; ++kk) {
-                    // dK += dS^T Q: dS^T K-major [keys x queries], Q as MN-major B
-                    const uint64_t a = sw128_desc(ds_addr + (kk >> 2) * kBlockBytes + (kk & 3) * 32,
-                                                  16, 1024);
-                    const uint64_t bd = sw128_desc(q_addr + kk * 2048, kBlockBytes, 1024);
-                    umma_bf16_ss(tmem + kColDK, a, bd, id_dk, (x > 0 || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < BN / 16; ++kk) {
+                        // dQ = dS K: dS^T read as an MN-major A (queries contiguous per key row)
+                        const uint64_t a = sw128_desc(ds_addr + kk * 2048, kBlockBytes, 1024);
+                        const uint64_t bd = sw128_desc(k_addr + kk * 2048, kBlockBytes, 1024);
+                        umma_bf16_ss(tmem + kColDP, a, bd, id_dq, kk > 0 ? 1u : 0u);
+                    }
+                    umma_commit(&bars[QD_EMPTY]);
+                    umma_commit(&bars[DQ_FULL]);
+                    ++x;
+                    ++g;
                 }
-                umma_commit(&bars[QD_EMPTY]);
-#pragma unroll
-                for (int kk = 0; kk < BN / 16; ++kk) {
-                    // dQ = dS K: dS^T read as an MN-major A (queries contiguous per key row)
-                    const uint64_t a = sw128_desc(ds_addr + kk * 2048, kBlockBytes, 1024);
-                    const uint64_t bd = sw128_desc(k_addr + kk * 2048, kBlockBytes, 1024);
-                    umma_bf16_ss(tmem + kColDP, a, bd, id_dq, kk > 0 ? 1u : 0u);
-                }
-                umma_commit(&bars[DQ_FULL]);
-                ++x;
+                if (!ok) break;
+                umma_commit(&bars[KV_EMPTY]);
+                umma_commit(&bars[ACC_FULL]);
+                ++n;
             }
-            umma_commit(&bars[ACC_FULL]);
             if (!ok) report_timeout(p);
             umma_commit(&bars[MMA_DONE]);
             if (!mbar_wait(&bars[MMA_DONE], 0)) report_timeout(p);
@@ -288,267 +579,225 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 3) {
         // -------------------------------------------------------------------- query stamps
         const bool use_ts = p.NB > 0;
-        QTileIter t(s, j0, p.W);
-        int x = 0;
-        while (t.next()) {
-            // the epilogue of the previous tile has read the staged stamps
-            if (x >= 1 && !warp_wait(&bars[P_FULL], (x - 1) & 1)) {
-                report_timeout(p);
-                break;
-            }
-            if (use_ts) {
-                const int i0 = t.qt * BM;
-                int64_t v[4];
-                int64_t mn[2] = {INT64_MAX, INT64_MAX}, mx[2] = {INT64_MIN, INT64_MIN};
+        UnitIter un(p, args.nkt, false);
+        int g = 0;
+        bool ok = true;
+        while (ok && un.next()) {
+            const SeqInfo &s = un.s;
+            QTileIter t(s, un.kt * BN, p.W);
+            while (t.next()) {
+                const int st = g & 1;
+                // the epilogue has finished with the stamps of tile g - 2
+                if (g >= 2 && !warp_wait(&bars[EPI_DONE + st], ((g >> 1) - 1) & 1)) {
+                    ok = false;
+                    break;
+                }
+                if (use_ts) {
+                    const int i0 = t.qt * BM;
 #pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    const int i = i0 + lane + 32 * q4;
-                    v[q4] = 0;
-                    if (i < s.L) {
-                        v[q4] = p.ts[s.start + clamp_pos(i, s.E)];
-                        mn[q4 >> 1] = min(mn[q4 >> 1], v[q4]);
-                        mx[q4 >> 1] = max(mx[q4 >> 1], v[q4]);
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        const int c = lane + 32 * q4, i = i0 + c;
+                        const bool in = i < s.L;
+                        const int64_t v = in ? p.ts[s.start + clamp_pos(i, s.E)] : 0;
+                        int64_t mn = in ? v : INT64_MAX, mx = in ? v : INT64_MIN;
+#pragma unroll
+                        for (int o = 16; o > 0; o >>= 1) {
+                            mn = min(mn, shfl_xor_i64(mn, o));
+                            mx = max(mx, shfl_xor_i64(mx, o));
+                        }
+                        const bool ok32 =
+                            mn > mx || (uint64_t)mx - (uint64_t)mn < (uint64_t)INT32_MAX;
+                        tsq[st * BM + c] = v;
+                        tsq32[st * BM + c] = (in && ok32) ? (int32_t)((uint64_t)v - (uint64_t)mn) : 0;
+                        if (lane == 0) {
+                            meta[st].tmin[q4] = mn;
+                            meta[st].tmax[q4] = mx;
+                            meta[st].ok32[q4] = ok32 ? 1 : 0;
+                        }
                     }
                 }
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh)
-#pragma unroll
-                    for (int o = 16; o > 0; o >>= 1) {
-                        mn[hh] = min(mn[hh], shfl_xor_i64(mn[hh], o));
-                        mx[hh] = max(mx[hh], shfl_xor_i64(mx[hh], o));
-                    }
-                int ok32[2];
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh)
-                    ok32[hh] = mn[hh] > mx[hh] ||
-                               (uint64_t)mx[hh] - (uint64_t)mn[hh] < (uint64_t)INT32_MAX;
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    const int c = lane + 32 * q4, hh = q4 >> 1;
-                    tsq[c] = v[q4];
-                    tsq32[c] = (i0 + c < s.L && ok32[hh])
-                                   ? (int32_t)((uint64_t)v[q4] - (uint64_t)mn[hh]) : 0;
-                }
-                if (lane == 0)
-#pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        meta->tmin[hh] = mn[hh];
-                        meta->tmax[hh] = mx[hh];
-                        meta->ok32[hh] = ok32[hh];
-                    }
+                warp_arrive(&bars[META_FULL + st]);
+                ++g;
             }
-            __syncwarp();
-            mbar_arrive(&bars[META_FULL]);
-            ++x;
         }
+        if (!ok) report_timeout(p);
     } else if (warp >= 4) {
         // -------------------------------------------------------------------- epilogue
-        const int wg = (warp - 4) >> 2;              // query columns [64 wg, 64 wg + 64)
+        const int wq = (warp - 4) >> 2;              // query columns [32 wq, 32 wq + 32)
         const int r = (warp & 3) * 32 + lane;        // key row in the tile == TMEM lane
-        const int j = j0 + r;
-        const bool key_in = j < s.L;
-        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-        const int pj = clamp_pos(j, s.E);
+        const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
         const bool use_ts = p.NB > 0, use_rel = p.R > 0;
-        const int64_t tsj = (use_ts && key_in) ? p.ts[s.start + pj] : 0;
-        const float *relp = rel_in_smem ? rels : p.rel;
         const bool lut_ok = *lut_valid != 0;
-        const int Em1 = s.E > 0 ? s.E - 1 : 0x7fffffff;   // p(i) = min(i, E-1) when E > 0
-        const uint32_t ds_row = sm_base + L::DS_OFF + wg * kBlockBytes + r * 128;
+        EpiBlock e;
+        e.t_s = tl + kColS + wq * QW;
+        e.t_dp = tl + kColDP + wq * QW;
+        e.t_a = tl + kColS + wq * QW;
+        e.ds_row = sm_base + L::YL_OFF + (wq >> 1) * kBlockBytes + r * 128;
+        e.ds_chunk0 = (wq & 1) * 4;
+        e.rsw = r & 7;
+        e.use_rel = use_rel;
+        e.use_ts = use_ts;
+        e.rel_in_smem = rel_in_smem;
+        e.relp = rel_in_smem ? rels : p.rel;
+        e.thr = thr;
+        e.tbs = tbs;
+        e.lut = lut;
+        e.tb_slot = tb_slot;
+        UnitIter un(p, args.nkt, false);
+        int n = 0, g = 0;
         bool ok = true;
-        QTileIter t(s, j0, p.W);
-        int x = 0;
-        while (t.next()) {
-            const int ih = t.qt * BM + wg * HALF;     // first query of this warpgroup's half
-            if (!warp_wait(&bars[META_FULL], x & 1) || !warp_wait(&bars[SD_FULL], x & 1)) {
-                ok = false;
-                break;
-            }
-            const bool full = tile_all_valid(ih, ih + HALF - 1, j0, j0 + BN - 1, s, p.W);
-            const uint64_t vmask = full ? ~0ull : col_valid_bits(j, ih, s, p.W);
-            // rel index p(i) - p(j) = rbase + c when no query of the half is a candidate
-            const int rbase = ih - pj;
-            const bool rdirect = __all_sync(0xffffffffu, !use_rel ||
-                                                              (ih + HALF - 1 < s.E && rbase >= 0 &&
-                                                               rbase + HALF - 1 <= p.R - 1));
-            HalfTime ht = {};
-            int tmode = 0;
-            if (use_ts) {
-                ht = half_time_setup(thr, p.n_thr, tbs, p.NB, key_in, tsj, meta->tmin[wg],
-                                     meta->tmax[wg], meta->ok32[wg] != 0, lut_ok, lut);
-                tmode = __reduce_max_sync(0xffffffffu, ht.my_mode);
-            }
-            float tsum_lo = 0.f, tsum_hi = 0.f;    // dS sums per bucket in modes 0/1
-            tc_fence_after();
-#pragma unroll 1
-            for (int ch = 0; ch < 2; ++ch) {
-                const int cb = ch * 32;
-                uint32_t rs[32], rd[32];
-                tmem_ld32(tmem + lane_base + kColS + wg * HALF + cb, rs);
-                tmem_ld32(tmem + lane_base + kColDP + wg * HALF + cb, rd);
-                tmem_wait_ld();
-                reg_fence(rs);
-                reg_fence(rd);
-                const uint32_t vbits = (uint32_t)(vmask >> cb);
-                uint32_t pa[16], pd[16];
-#pragma unroll
-                for (int c2 = 0; c2 < 16; ++c2) {
-                    float av[2], dv2[2];
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const int c = 2 * c2 + e, cc = cb + c;
-                        const int i = ih + cc;
-                        const bool valid = full || ((vbits >> c) & 1u);
-                        float bias = 0.f;
-                        int ri = -1, bk = -1;
-                        if (use_rel) {
-                            if (rdirect) {
-                                ri = rbase + cc;
-                            } else {
-                                ri = min(i, Em1) - pj;
-                                ri = ri < 0 ? 0 : (ri > p.R - 1 ? p.R - 1 : ri);
-                            }
-                            bias = relp[ri];
-                        }
-                        if (use_ts)
-                            bias += half_time_value(ht, tmode, tsq32[wg * HALF + cc],
-                                                    tsq[wg * HALF + cc], tsj, thr, p.n_thr, tbs,
-                                                    lut, &bk);
-                        // s = alpha q.k + b; SiLU(s) = s sigma(s); SiLU'(s) = sigma (1 + s (1 - sigma)).
-                        // sigma from the accurate exponential: table gradients sum dS over many
-                        // pairs and can cancel, so dS needs close to fp32 accuracy
-                        const float xs = fmaf(p.alpha, __uint_as_float(rs[c]), bias);
-                        const float sig = __fdividef(1.0f, 1.0f + __expf(-xs));
-                        const float silu = xs * sig;
-                        const float dsilu = sig * fmaf(xs, 1.0f - sig, 1.0f);
-                        const float a = valid ? silu * p.inv_N : 0.f;
-                        const float ds = valid ? __uint_as_float(rd[c]) * dsilu * p.inv_N : 0.f;
-                        av[e] = a;
-                        dv2[e] = ds;
-                        // table gradients
-                        if (valid) {
-                            if (use_rel) {
-                                if (rel_in_smem) atomicAdd(hrel + ri, ds);
-                                else atomicAdd(args.d_rel + ri, ds);
-                            }
-                            if (use_ts) {
-                                if (tmode <= 1) {
-                                    if (bk == ht.blo) tsum_lo += ds; else tsum_hi += ds;
-                                } else {
-                                    atomicAdd(htb + bk, ds);
-                                }
-                            }
-                        }
-                    }
-                    pa[c2] = pack_bf16x2(av[0], av[1]);
-                    pd[c2] = pack_bf16x2(dv2[0], dv2[1]);
+        while (ok && un.next()) {
+            const SeqInfo &s = un.s;
+            const int j0 = un.kt * BN, jw = j0 + (warp & 3) * 32;
+            KeyLane k;
+            k.j = j0 + r;
+            k.key_in = k.j < s.L;
+            k.pj = clamp_pos(k.j, s.E);
+            k.tsj = (use_ts && k.key_in) ? p.ts[s.start + k.pj] : 0;
+            k.sysA = k.sysB = k.cand = k.negs = k.fars = 0.f;
+            k.cur_b = 0;
+            k.run = 0.f;
+            e.Em1 = s.E > 0 ? s.E - 1 : 0x7fffffff;
+            QTileIter t(s, j0, p.W);
+            int x = 0;
+            while (t.next()) {
+                const int st = g & 1;
+                e.iq = t.qt * BM + wq * QW;
+                if (!warp_wait(&bars[META_FULL + st], (g >> 1) & 1) ||
+                    !warp_wait(&bars[SD_FULL], g & 1)) {
+                    ok = false;
+                    break;
                 }
-                // A^T over the first 32 of this warpgroup's S^T columns
-                tmem_st16(tmem + lane_base + kColS + wg * HALF + ch * 16, pa);
-                // dS^T row r, queries wg*64 + cb .. +31: 16-byte chunks (cb/8 .. cb/8+3), swizzled
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int chunk = (cb >> 3) + q;
-                    st_shared_v4(ds_row + ((chunk ^ (r & 7)) << 4), pd[4 * q], pd[4 * q + 1],
-                                 pd[4 * q + 2], pd[4 * q + 3]);
+                e.full = tile_all_valid(e.iq, e.iq + QW - 1, j0, j0 + BN - 1, s, p.W);
+                e.vbits = e.full ? 0xFFFFFFFFu : (uint32_t)col_valid_bits(k.j, e.iq, s, p.W);
+                // rel index p(i) - p(j) = rbase + c for every lane that has a valid pair in
+                // the block (lanes without one read the table at an in-range dummy base)
+                const bool idle = e.vbits == 0u;
+                const int rb = e.iq - k.pj;
+                e.rdirect = __all_sync(0xffffffffu,
+                                       !use_rel || (p.R >= QW &&
+                                                    (idle || (e.iq + QW - 1 < s.E && rb >= 0 &&
+                                                              rb + QW - 1 <= p.R - 1))));
+                e.rbase = idle ? 0 : rb;
+                e.tq32 = tsq32 + st * BM + wq * QW;
+                e.tq64 = tsq + st * BM + wq * QW;
+                HalfTime ht = {};
+                int tmode = 0;
+                if (use_ts) {
+                    ht = half_time_setup(thr, p.n_thr, tbs, p.NB, k.key_in, k.tsj,
+                                         meta[st].tmin[wq], meta[st].tmax[wq],
+                                         meta[st].ok32[wq] != 0, lut_ok, lut);
+                    tmode = __reduce_max_sync(0xffffffffu, ht.my_mode);
                 }
-            }
-            if (use_ts && tmode <= 1) {
-                if (tsum_lo != 0.f) atomicAdd(htb + ht.blo, tsum_lo);
-                if (tsum_hi != 0.f) atomicAdd(htb + min(ht.blo + 1, p.NB - 1), tsum_hi);
-            }
-            tmem_wait_st();
-            tc_fence_before();
-            fence_proxy_async_smem();
-            mbar_arrive(&bars[P_FULL]);
+                float t_lo = 0.f, t_hi = 0.f;
+                tc_fence_after();
+                if (tmode == 0) epi_block<0>(p, e, ht, k, t_lo, t_hi);
+                else if (tmode == 1) epi_block<1>(p, e, ht, k, t_lo, t_hi);
+                else if (tmode == 2) epi_block<2>(p, e, ht, k, t_lo, t_hi);
+                else epi_block<3>(p, e, ht, k, t_lo, t_hi);
+                tmem_wait_st();
+                tc_fence_before();
+                fence_proxy_async_smem();
+                warp_arrive(&bars[P_FULL]);
+                warp_arrive(&bars[EPI_DONE + st]);
+                if (use_ts && tmode == 1) {
+                    run_add(k, tb_slot, ht.blo, t_lo);
+                    run_add(k, tb_slot, ht.blo + 1, t_hi);
+                }
+                if (use_rel) flush_rel(p, k, e.iq, jw, e.Em1, hrel, args.d_rel, rel_in_smem);
 
-            // ---- dQ tile: lanes = query rows of this tile; columns split by warpgroup
-            if (!warp_wait(&bars[DQ_FULL], x & 1)) { ok = false; break; }
-            tc_fence_after();
-            {
-                const int i = t.qt * BM + r;
-                float *dqr = args.dq_acc + ((s.start + i) * (int64_t)p.H + h) * DQK;
-#pragma unroll 1
-                for (int c = wg * (DQK / 64); c < (wg + 1) * (DQK / 64); ++c) {
+                // ---- dQ tile: lanes = query rows of this tile; columns split by warpgroup
+                if (!warp_wait(&bars[DQ_FULL], g & 1)) { ok = false; break; }
+                tc_fence_after();
+                {
+                    constexpr int QC = DQK / 4;
+                    const int i = t.qt * BM + r;
                     uint32_t rq[32];
-                    tmem_ld32(tmem + lane_base + kColDP + c * 32, rq);
+                    if (QC == 32) {
+                        tmem_ld32(tl + kColDP + wq * QC, rq);
+                    } else {
+                        uint32_t (&r16)[16] = *reinterpret_cast<uint32_t(*)[16]>(rq);
+                        tmem_ld16(tl + kColDP + wq * QC, r16);
+                    }
                     tmem_wait_ld();
                     reg_fence(rq);
+                    tc_fence_before();
+                    warp_arrive(&bars[DQ_FREE]);
                     if (i < s.L) {
+                        float *dqr = args.dq_acc + ((s.start + i) * (int64_t)p.H + un.h) * DQK + wq * QC;
 #pragma unroll
-                        for (int q = 0; q < 8; ++q)
-                            red_add_v4(dqr + c * 32 + 4 * q, p.alpha * __uint_as_float(rq[4 * q]),
+                        for (int q = 0; q < QC / 4; ++q)
+                            red_add_v4(dqr + 4 * q, p.alpha * __uint_as_float(rq[4 * q]),
                                        p.alpha * __uint_as_float(rq[4 * q + 1]),
                                        p.alpha * __uint_as_float(rq[4 * q + 2]),
                                        p.alpha * __uint_as_float(rq[4 * q + 3]));
                     }
                 }
+                ++x;
+                ++g;
             }
-            tc_fence_before();
-            mbar_arrive(&bars[DQ_FREE]);
-            ++x;
-        }
-        // ---- dV and dK of the key rows (every key tile sees at least its diagonal tile)
-        if (ok && !warp_wait(&bars[ACC_FULL], 0)) ok = false;
-        if (ok && x == 0) {
-            if (key_in) {
-                __nv_bfloat16 *dvr = args.dv + ((s.start + j) * (int64_t)p.H + h) * DV;
-                __nv_bfloat16 *dkr = args.dk + ((s.start + j) * (int64_t)p.H + h) * DQK;
-                for (int c = wg * (DV / 2); c < (wg + 1) * (DV / 2); ++c) dvr[c] = __float2bfloat16_rn(0.f);
-                for (int c = wg * (DQK / 2); c < (wg + 1) * (DQK / 2); ++c) dkr[c] = __float2bfloat16_rn(0.f);
-            }
-        } else if (ok) {
+            if (!ok) break;
+            if (use_ts && k.run != 0.f) red_add(tb_slot + k.cur_b, k.run);
+            // ---- dV and dK of the key rows (every key tile sees at least its diagonal tile)
+            if (!warp_wait(&bars[ACC_FULL], n & 1)) { ok = false; break; }
             tc_fence_after();
-            __nv_bfloat16 *dvr = args.dv + ((s.start + j) * (int64_t)p.H + h) * DV;
-            __nv_bfloat16 *dkr = args.dk + ((s.start + j) * (int64_t)p.H + h) * DQK;
-#pragma unroll 1
-            for (int c = wg * (DV / 64); c < (wg + 1) * (DV / 64); ++c) {
-                uint32_t ra[32];
-                tmem_ld32(tmem + lane_base + kColDV + c * 32, ra);
+            {
+                constexpr int VC = DV / 4, KC = DQK / 4;
+                uint32_t ra[32], rk[32];
+                if (VC == 32) {
+                    tmem_ld32(tl + kColDV + wq * VC, ra);
+                } else {
+                    uint32_t (&r16)[16] = *reinterpret_cast<uint32_t(*)[16]>(ra);
+                    tmem_ld16(tl + kColDV + wq * VC, r16);
+                }
+                if (KC == 32) {
+                    tmem_ld32(tl + kColDK + wq * KC, rk);
+                } else {
+                    uint32_t (&r16)[16] = *reinterpret_cast<uint32_t(*)[16]>(rk);
+                    tmem_ld16(tl + kColDK + wq * KC, r16);
+                }
                 tmem_wait_ld();
                 reg_fence(ra);
-                if (key_in) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(dvr + c * 32);
+                reg_fence(rk);
+                tc_fence_before();
+                warp_arrive(&bars[ACC_FREE]);
+                if (k.key_in) {
+                    const int64_t row = (s.start + k.j) * (int64_t)p.H + un.h;
+                    const float sv = x > 0 ? 1.0f : 0.f, sk = x > 0 ? p.alpha : 0.f;
+                    uint4 *dvp = reinterpret_cast<uint4 *>(args.dv + row * DV + wq * VC);
+                    uint4 *dkp = reinterpret_cast<uint4 *>(args.dk + row * DQK + wq * KC);
 #pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        dst[q] = make_uint4(
-                            pack_bf16x2(__uint_as_float(ra[8 * q]), __uint_as_float(ra[8 * q + 1])),
-                            pack_bf16x2(__uint_as_float(ra[8 * q + 2]), __uint_as_float(ra[8 * q + 3])),
-                            pack_bf16x2(__uint_as_float(ra[8 * q + 4]), __uint_as_float(ra[8 * q + 5])),
-                            pack_bf16x2(__uint_as_float(ra[8 * q + 6]), __uint_as_float(ra[8 * q + 7])));
+                    for (int q = 0; q < VC / 8; ++q)
+                        dvp[q] = make_uint4(
+                            pack_bf16x2(sv * __uint_as_float(ra[8 * q]), sv * __uint_as_float(ra[8 * q + 1])),
+                            pack_bf16x2(sv * __uint_as_float(ra[8 * q + 2]), sv * __uint_as_float(ra[8 * q + 3])),
+                            pack_bf16x2(sv * __uint_as_float(ra[8 * q + 4]), sv * __uint_as_float(ra[8 * q + 5])),
+                            pack_bf16x2(sv * __uint_as_float(ra[8 * q + 6]), sv * __uint_as_float(ra[8 * q + 7])));
+#pragma unroll
+                    for (int q = 0; q < KC / 8; ++q)
+                        dkp[q] = make_uint4(
+                            pack_bf16x2(sk * __uint_as_float(rk[8 * q]), sk * __uint_as_float(rk[8 * q + 1])),
+                            pack_bf16x2(sk * __uint_as_float(rk[8 * q + 2]), sk * __uint_as_float(rk[8 * q + 3])),
+                            pack_bf16x2(sk * __uint_as_float(rk[8 * q + 4]), sk * __uint_as_float(rk[8 * q + 5])),
+                            pack_bf16x2(sk * __uint_as_float(rk[8 * q + 6]), sk * __uint_as_float(rk[8 * q + 7])));
                 }
             }
-#pragma unroll 1
-            for (int c = wg * (DQK / 64); c < (wg + 1) * (DQK / 64); ++c) {
-                uint32_t ra[32];
-                tmem_ld32(tmem + lane_base + kColDK + c * 32, ra);
-                tmem_wait_ld();
-                reg_fence(ra);
-                if (key_in) {
-                    const float al = p.alpha;
-                    uint4 *dst = reinterpret_cast<uint4 *>(dkr + c * 32);
-#pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        dst[q] = make_uint4(
-                            pack_bf16x2(al * __uint_as_float(ra[8 * q]), al * __uint_as_float(ra[8 * q + 1])),
-                            pack_bf16x2(al * __uint_as_float(ra[8 * q + 2]), al * __uint_as_float(ra[8 * q + 3])),
-                            pack_bf16x2(al * __uint_as_float(ra[8 * q + 4]), al * __uint_as_float(ra[8 * q + 5])),
-                            pack_bf16x2(al * __uint_as_float(ra[8 * q + 6]), al * __uint_as_float(ra[8 * q + 7])));
-                }
-            }
-        } else {
-            report_timeout(p);
+            ++n;
         }
+        if (!ok) report_timeout(p);
     }
 
     tc_fence_before();
+    __threadfence();   // reductions into the slot row are complete before it is read back
     __syncthreads();
-    // flush the table-gradient histograms
+    // fold this CTA's table-gradient histograms into the outputs
     if (rel_in_smem)
         for (int x = threadIdx.x; x < p.R; x += kThreads)
             if (hrel[x] != 0.f) atomicAdd(args.d_rel + x, hrel[x]);
-    for (int x = threadIdx.x; x < p.NB; x += kThreads)
-        if (htb[x] != 0.f) atomicAdd(args.d_tb + x, htb[x]);
+    for (int x = threadIdx.x; x < p.NB; x += kThreads) {
+        const float v = ld_cg(tb_slot + x);
+        if (v != 0.f) atomicAdd(args.d_tb + x, v);
+    }
     if (warp == 2) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
@@ -559,11 +808,16 @@ template <int DQK, int DV>
 cudaError_t launch_bwd(const BwdTcArgs &a, cudaStream_t st)
 {
     using L = BwdLayout<DQK, DV>;
+    static_assert(L::ALLOC <= 232448, "shared memory layout exceeds the per-CTA limit");
     auto kern = bwd_tc_kernel<DQK, DV>;
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
     if (e != cudaSuccess) return e;
-    dim3 grid((a.p.N + BN - 1) / BN, a.p.B, a.p.H);
+    const int64_t units = (int64_t)a.nkt * a.p.B * a.p.H;
+    int grid = num_sms();
+    if (grid > kBwdMaxCtas) grid = kBwdMaxCtas;
+    if (units < grid) grid = (int)units;
+    if (grid <= 0) return cudaSuccess;
     kern<<<grid, kThreads, L::ALLOC, st>>>(a);
     return cudaGetLastError();
 }
@@ -574,7 +828,7 @@ bool tc_bwd_supported(int dqk, int dv, int64_t T) { return tc_fwd_supported(dqk,
 
 cudaError_t launch_tc_bwd(const DevParams &p, const void *q, const void *k, const void *v,
                           const void *dy_bf16, float *dq_acc, void *dk, void *dv, float *d_rel,
-                          float *d_tb, cudaStream_t st)
+                          float *d_tb, float *tb_slots, cudaStream_t st)
 {
     BwdTcArgs a;
     std::memset(&a, 0, sizeof(a));
@@ -584,6 +838,8 @@ cudaError_t launch_tc_bwd(const DevParams &p, const void *q, const void *k, cons
     a.dv = reinterpret_cast<__nv_bfloat16 *>(dv);
     a.d_rel = d_rel;
     a.d_tb = d_tb;
+    a.tb_slots = tb_slots;
+    a.nkt = (p.N + BN - 1) / BN;
     const void *dy_lo = reinterpret_cast<const char *>(dy_bf16) + (size_t)p.T * p.D * 2;
     if (!encode_tmap_bf16(&a.tq, q, p.dqk, p.H, p.T) || !encode_tmap_bf16(&a.tk, k, p.dqk, p.H, p.T) ||
         !encode_tmap_bf16(&a.tv, v, p.dv, p.H, p.T) ||

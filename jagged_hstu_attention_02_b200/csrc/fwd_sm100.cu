@@ -610,6 +610,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
 }
 
+}  // namespace
 
 int num_sms()
 {
@@ -624,6 +625,8 @@ int num_sms()
     }
     return n;
 }
+
+namespace {
 
 template <int DQK, int DV>
 cudaError_t launch_tc(const FwdTcArgs &a, bool split, cudaStream_t st)

@@ -34,12 +34,18 @@ bool tc_fwd_supported(int dqk, int dv, int64_t T);
 cudaError_t launch_tc_fwd(const DevParams &p, const void *q, const void *k, const void *v,
                           float *y, bool training, cudaStream_t st);
 
+// Multiprocessors of the current device (cached after the first query).
+int num_sms();
+
 // tcgen05 backward attention (bf16): dQ added into an fp32 accumulator (zeroed by the
 // caller), dK/dV written, table gradients added into d_rel/d_tb (zeroed by the caller).
+// tb_slots is scratch of kBwdMaxCtas * kMaxTimeBuckets floats (no initial contents).
+constexpr int kBwdMaxCtas = 1024;
 bool tc_bwd_supported(int dqk, int dv, int64_t T);
 cudaError_t launch_tc_bwd(const DevParams &p, const void *q, const void *k, const void *v,
-                          const void *dy_bf16 /* hi, then lo at + T*D */, float *dq_acc, void *dk, void *dv, float *d_rel,
-                          float *d_tb, cudaStream_t st);
+                          const void *dy_bf16 /* hi, then lo at + T*D */, float *dq_acc,
+                          void *dk, void *dv, float *d_rel, float *d_tb, float *tb_slots,
+                          cudaStream_t st);
 
 // [T, H, d] bf16 row-major as a 3-D TMA tensor (d, H, T): box 64 x 1 x 128, 128-byte swizzle.
 bool encode_tmap_bf16(CUtensorMap *m, const void *base, int d, int H, int64_t T);
