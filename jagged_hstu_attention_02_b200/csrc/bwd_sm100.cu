@@ -49,6 +49,7 @@ constexpr int QW = 32;                  // query columns per epilogue warpgroup
 constexpr int kEpiWarps = 16;
 constexpr int kThreads = 128 + 32 * kEpiWarps;
 constexpr int kRelSmemMax = 2048;
+constexpr int kRelGuard = 32;           // zero entries on both sides of the shared rel table
 constexpr uint32_t kTmemCols = 512;
 constexpr int kBlockBytes = 128 * 128;
 // TMEM columns: S^T -> A^T [0,128); dP^T -> dQ tile [128,256); dV [256,384); dK [384,512)
@@ -89,7 +90,7 @@ struct BwdLayout {
     static constexpr int THR_OFF = LUT_OFF + kLutCells * 8;
     static constexpr int TB_OFF = THR_OFF + 8 * kMaxTimeBuckets;
     static constexpr int REL_OFF = TB_OFF + 4 * kMaxTimeBuckets;
-    static constexpr int HREL_OFF = REL_OFF + 4 * kRelSmemMax;
+    static constexpr int HREL_OFF = REL_OFF + 4 * (kRelSmemMax + 2 * kRelGuard);
     static constexpr int TOTAL = HREL_OFF + 4 * kRelSmemMax;
     static constexpr int ALLOC = TOTAL + 1024;
     static_assert(NUM_BARS <= 16, "barrier area");
@@ -213,9 +214,9 @@ struct EpiBlock {
     uint32_t ds_row;              // smem address of this key's dS^T row (first 16-byte chunk)
     int ds_chunk0, rsw;           // first chunk of the block in the row, swizzle (row & 7)
     int iq;                       // first query of the block
-    int rbase;                    // p(iq) - p(j) when rdirect
+    int rbase;                    // p(iq) - p(j) in DIRECT blocks
     int Em1;                      // p(i) = min(i, Em1)
-    bool full, rdirect, use_rel, use_ts, rel_in_smem;
+    bool full, use_rel, use_ts, rel_in_smem;
     uint32_t vbits;               // valid queries of this key (bit c <-> query iq + c)
     const int32_t *tq32;          // the block's query stamps relative to the quarter minimum
     const int64_t *tq64;          // and absolute
@@ -226,7 +227,10 @@ struct EpiBlock {
     float *tb_slot;
 };
 
-template <int TM>
+// DIRECT: every valid pair of the block has rel index p(i) - p(j) = rbase + c in [0, R)
+// (no candidate row, no clamping), and the table sits in shared memory with a guard band
+// that keeps the reads of masked pairs (at most 31 entries off) in bounds.
+template <int TM, bool DIRECT>
 __device__ __forceinline__ void epi_block(const DevParams &p, const EpiBlock &e,
                                           const HalfTime &ht, KeyLane &k, float &t_lo,
                                           float &t_hi)
@@ -283,7 +287,7 @@ __device__ __forceinline__ void epi_block(const DevParams &p, const EpiBlock &e,
                 }
                 int rraw = 0, ri = 0;
                 if (e.use_rel) {
-                    if (e.rdirect) {
+                    if (DIRECT) {
                         ri = e.rbase + cc;
                     } else {
                         rraw = min(i, e.Em1) - k.pj;
@@ -305,7 +309,7 @@ __device__ __forceinline__ void epi_block(const DevParams &p, const EpiBlock &e,
                 // ---- rel gradient: shift the diagonal sums one lane down, add this column
                 if (e.use_rel) {
                     float vd = ds;
-                    if (!e.rdirect) {
+                    if (!DIRECT) {
                         if (i > e.Em1) {              // candidate row (warp-uniform)
                             k.cand += ds;
                             vd = 0.f;
@@ -408,7 +412,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     LutEntry *lut = reinterpret_cast<LutEntry *>(sm + L::LUT_OFF);
     uint64_t *thr = reinterpret_cast<uint64_t *>(sm + L::THR_OFF);
     float *tbs = reinterpret_cast<float *>(sm + L::TB_OFF);
-    float *rels = reinterpret_cast<float *>(sm + L::REL_OFF);
+    float *rels = reinterpret_cast<float *>(sm + L::REL_OFF) + kRelGuard;
     float *hrel = reinterpret_cast<float *>(sm + L::HREL_OFF);
     float *tb_slot = args.tb_slots + (size_t)blockIdx.x * kMaxTimeBuckets;
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -430,11 +434,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         tb_slot[x] = 0.f;
     }
     const bool rel_in_smem = p.R <= kRelSmemMax;
-    if (rel_in_smem)
+    if (rel_in_smem) {
         for (int x = threadIdx.x; x < p.R; x += kThreads) {
             rels[x] = p.rel[x];
             hrel[x] = 0.f;
         }
+        for (int x = threadIdx.x; x < kRelGuard; x += kThreads) {
+            rels[-1 - x] = 0.f;
+            rels[p.R + x] = 0.f;
+        }
+    }
     __threadfence();   // the zeroed slot row is in place before any reduction into it
     __syncthreads();
     if (p.NB > 0) build_lut(thr, p.n_thr, lut, lut_valid);
@@ -670,41 +679,68 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 e.full = tile_all_valid(e.iq, e.iq + QW - 1, j0, j0 + BN - 1, s, p.W);
                 e.vbits = e.full ? 0xFFFFFFFFu : (uint32_t)col_valid_bits(k.j, e.iq, s, p.W);
-                // rel index p(i) - p(j) = rbase + c for every lane that has a valid pair in
-                // the block (lanes without one read the table at an in-range dummy base)
-                const bool idle = e.vbits == 0u;
-                const int rb = e.iq - k.pj;
-                e.rdirect = __all_sync(0xffffffffu,
-                                       !use_rel || (p.R >= QW &&
-                                                    (idle || (e.iq + QW - 1 < s.E && rb >= 0 &&
-                                                              rb + QW - 1 <= p.R - 1))));
-                e.rbase = idle ? 0 : rb;
-                e.tq32 = tsq32 + st * BM + wq * QW;
-                e.tq64 = tsq + st * BM + wq * QW;
-                HalfTime ht = {};
-                int tmode = 0;
-                if (use_ts) {
-                    ht = half_time_setup(thr, p.n_thr, tbs, p.NB, k.key_in, k.tsj,
-                                         meta[st].tmin[wq], meta[st].tmax[wq],
-                                         meta[st].ok32[wq] != 0, lut_ok, lut);
-                    tmode = __reduce_max_sync(0xffffffffu, ht.my_mode);
+                const uint32_t vb = e.vbits;
+                const bool idle = vb == 0u;
+                if (!__any_sync(0xffffffffu, !idle)) {
+                    // no valid pair in the block: A and dS are zero, no table gradient
+                    const uint32_t z[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+                    tmem_st8(e.t_a, z);
+                    tmem_st8(e.t_a + 8, z);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        st_shared_v4(e.ds_row + (((e.ds_chunk0 + q) ^ e.rsw) << 4), 0u, 0u, 0u, 0u);
+                    tmem_wait_st();
+                    tc_fence_before();
+                    fence_proxy_async_smem();
+                    warp_arrive(&bars[P_FULL]);
+                    warp_arrive(&bars[EPI_DONE + st]);
+                } else {
+                    // DIRECT blocks: every valid pair has rel index p(i) - p(j) = rbase + c
+                    // within the table and no candidate row (lanes without a valid pair
+                    // read the guarded table at base 0)
+                    const int fc = e.Em1 - e.iq + 1;           // first candidate column
+                    const uint32_t candbits = fc >= QW ? 0u : (fc <= 0 ? ~0u : (~0u << fc));
+                    const int rb = e.iq - k.pj;
+                    const int c_lo = __ffs(vb) - 1, c_hi = 31 - __clz(vb);
+                    const bool lane_direct =
+                        idle || ((vb & candbits) == 0u && rb + c_lo >= 0 && rb + c_hi <= p.R - 1);
+                    const bool direct =
+                        !use_rel || (rel_in_smem && __all_sync(0xffffffffu, lane_direct));
+                    e.rbase = idle ? 0 : rb;
+                    e.tq32 = tsq32 + st * BM + wq * QW;
+                    e.tq64 = tsq + st * BM + wq * QW;
+                    HalfTime ht = {};
+                    int tmode = 0;
+                    if (use_ts) {
+                        ht = half_time_setup(thr, p.n_thr, tbs, p.NB, k.key_in, k.tsj,
+                                             meta[st].tmin[wq], meta[st].tmax[wq],
+                                             meta[st].ok32[wq] != 0, lut_ok, lut);
+                        tmode = __reduce_max_sync(0xffffffffu, ht.my_mode);
+                    }
+                    float t_lo = 0.f, t_hi = 0.f;
+                    tc_fence_after();
+                    if (direct) {
+                        if (tmode == 0) epi_block<0, true>(p, e, ht, k, t_lo, t_hi);
+                        else if (tmode == 1) epi_block<1, true>(p, e, ht, k, t_lo, t_hi);
+                        else if (tmode == 2) epi_block<2, true>(p, e, ht, k, t_lo, t_hi);
+                        else epi_block<3, false>(p, e, ht, k, t_lo, t_hi);
+                    } else {
+                        if (tmode == 0) epi_block<0, false>(p, e, ht, k, t_lo, t_hi);
+                        else if (tmode == 1) epi_block<1, false>(p, e, ht, k, t_lo, t_hi);
+                        else if (tmode == 2) epi_block<2, false>(p, e, ht, k, t_lo, t_hi);
+                        else epi_block<3, false>(p, e, ht, k, t_lo, t_hi);
+                    }
+                    tmem_wait_st();
+                    tc_fence_before();
+                    fence_proxy_async_smem();
+                    warp_arrive(&bars[P_FULL]);
+                    warp_arrive(&bars[EPI_DONE + st]);
+                    if (use_ts && tmode == 1) {
+                        run_add(k, tb_slot, ht.blo, t_lo);
+                        run_add(k, tb_slot, ht.blo + 1, t_hi);
+                    }
+                    if (use_rel) flush_rel(p, k, e.iq, jw, e.Em1, hrel, args.d_rel, rel_in_smem);
                 }
-                float t_lo = 0.f, t_hi = 0.f;
-                tc_fence_after();
-                if (tmode == 0) epi_block<0>(p, e, ht, k, t_lo, t_hi);
-                else if (tmode == 1) epi_block<1>(p, e, ht, k, t_lo, t_hi);
-                else if (tmode == 2) epi_block<2>(p, e, ht, k, t_lo, t_hi);
-                else epi_block<3>(p, e, ht, k, t_lo, t_hi);
-                tmem_wait_st();
-                tc_fence_before();
-                fence_proxy_async_smem();
-                warp_arrive(&bars[P_FULL]);
-                warp_arrive(&bars[EPI_DONE + st]);
-                if (use_ts && tmode == 1) {
-                    run_add(k, tb_slot, ht.blo, t_lo);
-                    run_add(k, tb_slot, ht.blo + 1, t_hi);
-                }
-                if (use_rel) flush_rel(p, k, e.iq, jw, e.Em1, hrel, args.d_rel, rel_in_smem);
 
                 // ---- dQ tile: lanes = query rows of this tile; columns split by warpgroup
                 if (!warp_wait(&bars[DQ_FULL], g & 1)) { ok = false; break; }
