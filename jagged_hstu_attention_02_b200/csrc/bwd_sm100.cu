@@ -47,7 +47,8 @@ namespace {
 constexpr int BM = 128, BN = 128;
 constexpr int QW = 32;                  // query columns per epilogue warpgroup
 constexpr int kEpiWarps = 16;
-constexpr int kThreads = 128 + 32 * kEpiWarps;
+constexpr int kEpiWarp0 = 3;            // warps 0-2: TMA, MMA, TMEM owner + query stamps
+constexpr int kThreads = 32 * (kEpiWarp0 + kEpiWarps);
 constexpr int kRelSmemMax = 2048;
 constexpr int kRelGuard = 32;           // zero entries on both sides of the shared rel table
 constexpr uint32_t kTmemCols = 512;
@@ -172,9 +173,26 @@ __device__ __forceinline__ void red_add_v4(float *addr, float a, float b, float 
                  : "memory");
 }
 
+// No "memory" clobber: the target never aliases what the epilogue loads, and a clobber
+// would stop the compiler from overlapping the loads of neighbouring pairs.  Volatile asm
+// keeps its order relative to the fence_gpu() that precedes the read-back.
 __device__ __forceinline__ void red_add(float *addr, float a)
 {
-    asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(a) : "memory");
+    asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(a));
+}
+
+// red_add when `pred` holds, as a predicated instruction (no branch).  A zero value adds
+// nothing, so it is not tested.
+__device__ __forceinline__ void red_add_if(float *addr, float a, bool pred)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %2, 0;\n\t@p red.global.add.f32 [%0], %1;\n\t}" ::"l"(addr),
+        "f"(a), "r"((int)pred));
+}
+
+__device__ __forceinline__ void fence_gpu()
+{
+    asm volatile("fence.acq_rel.gpu;" ::: "memory");
 }
 
 __device__ __forceinline__ float ld_cg(const float *addr)
@@ -210,7 +228,7 @@ struct KeyLane {
 // and accumulates the table gradients into the lane state.  TM is the warp-uniform time
 // mode of half_time_setup (0 when there is no time bias).
 struct EpiBlock {
-    uint32_t t_s, t_dp, t_a;      // TMEM addresses of the block's S^T, dP^T and A^T columns
+    uint32_t t_s, t_dp;           // TMEM addresses of the block's S^T (then A^T) and dP^T
     uint32_t ds_row;              // smem address of this key's dS^T row (first 16-byte chunk)
     int ds_chunk0, rsw;           // first chunk of the block in the row, swizzle (row & 7)
     int iq;                       // first query of the block
@@ -235,6 +253,8 @@ __device__ __forceinline__ void epi_block(const DevParams &p, const EpiBlock &e,
                                           const HalfTime &ht, KeyLane &k, float &t_lo,
                                           float &t_hi)
 {
+    // The body is free of branches (selects and predicated reductions only), so the
+    // compiler can overlap the loads and the arithmetic of neighbouring pairs.
     const int lane = threadIdx.x & 31;
     if (TM == 0 && e.use_ts && k.key_in) {
         if (ht.blo != k.cur_b) {
@@ -243,25 +263,28 @@ __device__ __forceinline__ void epi_block(const DevParams &p, const EpiBlock &e,
             k.run = 0.f;
         }
     }
-#pragma unroll
-    for (int hf = 0; hf < 2; ++hf) {
-        uint32_t rs[16], rd[16];
-        tmem_ld16(e.t_s + hf * 16, rs);
-        tmem_ld16(e.t_dp + hf * 16, rd);
+    const bool lane0 = lane == 0;
+    const int src = (lane + 31) & 31;
+#pragma unroll 1
+    for (int ch = 0; ch < 4; ++ch) {
+        // 8 query columns: one 16-byte chunk of the dS^T row, 4 TMEM columns of A^T
+        uint32_t rs[8], rd[8];
+        tmem_ld8(e.t_s + ch * 8, rs);
+        tmem_ld8(e.t_dp + ch * 8, rd);
         tmem_wait_ld();
         reg_fence(rs);
         reg_fence(rd);
-        uint32_t pa[8], pd[8];
+        uint32_t pa[4], pd[4];
 #pragma unroll
-        for (int c2 = 0; c2 < 8; ++c2) {
+        for (int c2 = 0; c2 < 4; ++c2) {
             float av[2], dv2[2];
 #pragma unroll
             for (int q = 0; q < 2; ++q) {
-                const int c = 2 * c2 + q, cc = hf * 16 + c;
+                const int c = 2 * c2 + q, cc = ch * 8 + c;
                 const int i = e.iq + cc;
-                const bool valid = e.full || ((e.vbits >> cc) & 1u);
+                const bool valid = (e.vbits >> cc) & 1u;
                 // ---- bias
-                float bias = 0.f;
+                float bias;
                 int bk = 0;
                 if (TM == 0) {
                     bias = ht.tb_lo;
@@ -271,30 +294,24 @@ __device__ __forceinline__ void epi_block(const DevParams &p, const EpiBlock &e,
                     bias = hi ? ht.tb_hi : ht.tb_lo;
                     bk = hi ? 1 : 0;
                 } else if (TM == 2) {
-                    if (ht.lane_const) {
-                        bias = ht.tb_lo;
-                        bk = ht.blo;
-                    } else {
-                        const int32_t d = ht.t_rel - e.tq32[cc];
-                        uint32_t dt = (uint32_t)(d < 0 ? -d : d);
-                        dt = min(dt, (uint32_t)INT32_MAX - 1u);
-                        bk = lut_bucket(e.lut, dt);
-                        bias = e.tbs[bk];
-                    }
+                    const int32_t d = ht.t_rel - e.tq32[cc];
+                    uint32_t dt = (uint32_t)(d < 0 ? -d : d);
+                    dt = min(dt, (uint32_t)INT32_MAX - 1u);
+                    const int b = lut_bucket(e.lut, dt);
+                    bk = ht.lane_const ? ht.blo : b;
+                    bias = ht.lane_const ? ht.tb_lo : e.tbs[b];
                 } else {
                     bk = bucket_search(e.thr, p.n_thr, abs_diff_u64(k.tsj, e.tq64[cc]));
                     bias = e.tbs[bk];
                 }
-                int rraw = 0, ri = 0;
-                if (e.use_rel) {
-                    if (DIRECT) {
-                        ri = e.rbase + cc;
-                    } else {
-                        rraw = min(i, e.Em1) - k.pj;
-                        ri = rraw < 0 ? 0 : (rraw > p.R - 1 ? p.R - 1 : rraw);
-                    }
-                    bias += e.relp[ri];
+                int rraw = 0, ri;
+                if (DIRECT) {
+                    ri = e.rbase + cc;
+                } else {
+                    rraw = min(i, e.Em1) - k.pj;
+                    ri = rraw < 0 ? 0 : (rraw > p.R - 1 ? p.R - 1 : rraw);
                 }
+                bias += e.relp[ri];
                 // ---- s = alpha q.k + b; SiLU(s) = s sigma(s); SiLU'(s) = sigma (1 + s (1 - sigma)).
                 // sigma from the accurate exponential: table gradients sum dS over many pairs
                 // and can cancel, so dS needs close to fp32 accuracy
@@ -307,48 +324,37 @@ __device__ __forceinline__ void epi_block(const DevParams &p, const EpiBlock &e,
                 av[q] = a;
                 dv2[q] = ds;
                 // ---- rel gradient: shift the diagonal sums one lane down, add this column
-                if (e.use_rel) {
-                    float vd = ds;
-                    if (!DIRECT) {
-                        if (i > e.Em1) {              // candidate row (warp-uniform)
-                            k.cand += ds;
-                            vd = 0.f;
-                        } else if (rraw != ri) {
-                            if (rraw < 0) k.negs += ds; else k.fars += ds;
-                            vd = 0.f;
-                        }
-                    }
-                    const float ain = __shfl_sync(0xffffffffu, k.sysA, (lane + 31) & 31);
-                    const float bin = __shfl_sync(0xffffffffu, k.sysB, (lane + 31) & 31);
-                    k.sysB = lane == 0 ? ain : bin;
-                    k.sysA = (lane == 0 ? 0.f : ain) + vd;
+                float vd = ds;
+                if (!DIRECT) {
+                    const bool candc = i > e.Em1;            // candidate row (warp-uniform)
+                    const bool clamped = rraw != ri;
+                    k.cand += candc ? ds : 0.f;
+                    k.negs += (!candc && clamped && rraw < 0) ? ds : 0.f;
+                    k.fars += (!candc && clamped && rraw >= 0) ? ds : 0.f;
+                    vd = (candc || clamped) ? 0.f : ds;
                 }
+                const float ain = __shfl_sync(0xffffffffu, k.sysA, src);
+                const float bin = __shfl_sync(0xffffffffu, k.sysB, src);
+                k.sysB = lane0 ? ain : bin;
+                k.sysA = (lane0 ? 0.f : ain) + vd;
                 // ---- time gradient
-                if (e.use_ts) {
-                    if (TM == 0) {
-                        k.run += ds;
-                    } else if (TM == 1) {
-                        if (bk) t_hi += ds; else t_lo += ds;
-                    } else if (valid) {
-                        if (bk != k.cur_b) {
-                            if (k.run != 0.f) red_add(e.tb_slot + k.cur_b, k.run);
-                            k.cur_b = bk;
-                            k.run = 0.f;
-                        }
-                        k.run += ds;
-                    }
+                if (TM == 0) {
+                    k.run += ds;
+                } else if (TM == 1) {
+                    t_hi += bk ? ds : 0.f;
+                    t_lo += bk ? 0.f : ds;
+                } else {
+                    const bool chg = valid && bk != k.cur_b;
+                    red_add_if(e.tb_slot + k.cur_b, k.run, chg && e.use_ts);
+                    k.cur_b = chg ? bk : k.cur_b;
+                    k.run = (chg ? 0.f : k.run) + ds;
                 }
             }
             pa[c2] = pack_bf16x2(av[0], av[1]);
             pd[c2] = pack_bf16x2(dv2[0], dv2[1]);
         }
-        tmem_st8(e.t_a + hf * 8, pa);
-#pragma unroll
-        for (int q = 0; q < 2; ++q) {
-            const int chunk = e.ds_chunk0 + hf * 2 + q;
-            st_shared_v4(e.ds_row + ((chunk ^ e.rsw) << 4), pd[4 * q], pd[4 * q + 1],
-                         pd[4 * q + 2], pd[4 * q + 3]);
-        }
+        tmem_st4(e.t_s + ch * 4, pa);
+        st_shared_v4(e.ds_row + (((e.ds_chunk0 + ch) ^ e.rsw) << 4), pd[0], pd[1], pd[2], pd[3]);
     }
 }
 
@@ -392,6 +398,42 @@ __device__ __forceinline__ void run_add(KeyLane &k, float *slot, int b, float v)
     } else {
         k.run += v;
     }
+}
+
+// Reads NC fp32 columns of this lane's TMEM row starting at taddr, in pieces of up to 32.
+template <int NC, typename F>
+__device__ __forceinline__ void tmem_row_foreach(uint32_t taddr, F &&f)
+{
+    if constexpr (NC >= 32) {
+#pragma unroll
+        for (int cq = 0; cq < NC / 32; ++cq) {
+            uint32_t v[32];
+            tmem_ld32(taddr + cq * 32, v);
+            tmem_wait_ld();
+            reg_fence(v);
+            f(cq * 32, v);
+        }
+    } else {
+        uint32_t v[16];
+        tmem_ld16(taddr, v);
+        tmem_wait_ld();
+        reg_fence(v);
+        f(0, v);
+    }
+}
+
+// Stores n fp32 values (times sc) as bf16, 8 per 16-byte store.
+template <int N>
+__device__ __forceinline__ void store_bf16_row(__nv_bfloat16 *dst, const uint32_t (&v)[N], float sc)
+{
+    uint4 *dp = reinterpret_cast<uint4 *>(dst);
+#pragma unroll
+    for (int q = 0; q < N / 8; ++q)
+        dp[q] = make_uint4(
+            pack_bf16x2(sc * __uint_as_float(v[8 * q]), sc * __uint_as_float(v[8 * q + 1])),
+            pack_bf16x2(sc * __uint_as_float(v[8 * q + 2]), sc * __uint_as_float(v[8 * q + 3])),
+            pack_bf16x2(sc * __uint_as_float(v[8 * q + 4]), sc * __uint_as_float(v[8 * q + 5])),
+            pack_bf16x2(sc * __uint_as_float(v[8 * q + 6]), sc * __uint_as_float(v[8 * q + 7])));
 }
 
 template <int DQK, int DV>
@@ -585,7 +627,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             umma_commit(&bars[MMA_DONE]);
             if (!mbar_wait(&bars[MMA_DONE], 0)) report_timeout(p);
         }
-    } else if (warp == 3) {
+    } else if (warp == 2) {
         // -------------------------------------------------------------------- query stamps
         const bool use_ts = p.NB > 0;
         UnitIter un(p, args.nkt, false);
@@ -630,19 +672,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         if (!ok) report_timeout(p);
-    } else if (warp >= 4) {
+    } else if (warp >= kEpiWarp0) {
         // -------------------------------------------------------------------- epilogue
-        const int wq = (warp - 4) >> 2;              // query columns [32 wq, 32 wq + 32)
+        constexpr int kGroups = kEpiWarps / 4;        // warpgroups
+        constexpr int kQPer = 4 / kGroups;            // 32-query blocks per warp and tile
+        const int wg = (warp - kEpiWarp0) >> 2;      // query columns [128/kGroups * wg, ...)
         const int r = (warp & 3) * 32 + lane;        // key row in the tile == TMEM lane
         const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
         const bool use_ts = p.NB > 0, use_rel = p.R > 0;
         const bool lut_ok = *lut_valid != 0;
         EpiBlock e;
-        e.t_s = tl + kColS + wq * QW;
-        e.t_dp = tl + kColDP + wq * QW;
-        e.t_a = tl + kColS + wq * QW;
-        e.ds_row = sm_base + L::YL_OFF + (wq >> 1) * kBlockBytes + r * 128;
-        e.ds_chunk0 = (wq & 1) * 4;
         e.rsw = r & 7;
         e.use_rel = use_rel;
         e.use_ts = use_ts;
@@ -671,30 +710,34 @@ __global__ void __launch_bounds__(kThreads, 1)
             int x = 0;
             while (t.next()) {
                 const int st = g & 1;
-                e.iq = t.qt * BM + wq * QW;
                 if (!warp_wait(&bars[META_FULL + st], (g >> 1) & 1) ||
                     !warp_wait(&bars[SD_FULL], g & 1)) {
                     ok = false;
                     break;
                 }
-                e.full = tile_all_valid(e.iq, e.iq + QW - 1, j0, j0 + BN - 1, s, p.W);
-                e.vbits = e.full ? 0xFFFFFFFFu : (uint32_t)col_valid_bits(k.j, e.iq, s, p.W);
-                const uint32_t vb = e.vbits;
-                const bool idle = vb == 0u;
-                if (!__any_sync(0xffffffffu, !idle)) {
-                    // no valid pair in the block: A and dS are zero, no table gradient
-                    const uint32_t z[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-                    tmem_st8(e.t_a, z);
-                    tmem_st8(e.t_a + 8, z);
+#pragma unroll 1
+                for (int qq = 0; qq < kQPer; ++qq) {
+                    const int wq = wg * kQPer + qq;          // query columns [32 wq, 32 wq + 32)
+                    e.iq = t.qt * BM + wq * QW;
+                    e.t_s = tl + kColS + wq * QW;
+                    e.t_dp = tl + kColDP + wq * QW;
+                    e.ds_row = sm_base + L::YL_OFF + (wq >> 1) * kBlockBytes + r * 128;
+                    e.ds_chunk0 = (wq & 1) * 4;
+                    e.full = tile_all_valid(e.iq, e.iq + QW - 1, j0, j0 + BN - 1, s, p.W);
+                    e.vbits = e.full ? 0xFFFFFFFFu : (uint32_t)col_valid_bits(k.j, e.iq, s, p.W);
+                    const uint32_t vb = e.vbits;
+                    const bool idle = vb == 0u;
+                    if (!__any_sync(0xffffffffu, !idle)) {
+                        // no valid pair in the block: A and dS are zero, no table gradient
+                        const uint32_t z[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+                        tmem_st8(e.t_s, z);
+                        tmem_st8(e.t_s + 8, z);
 #pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        st_shared_v4(e.ds_row + (((e.ds_chunk0 + q) ^ e.rsw) << 4), 0u, 0u, 0u, 0u);
-                    tmem_wait_st();
-                    tc_fence_before();
-                    fence_proxy_async_smem();
-                    warp_arrive(&bars[P_FULL]);
-                    warp_arrive(&bars[EPI_DONE + st]);
-                } else {
+                        for (int q = 0; q < 4; ++q)
+                            st_shared_v4(e.ds_row + (((e.ds_chunk0 + q) ^ e.rsw) << 4), 0u, 0u,
+                                         0u, 0u);
+                        continue;
+                    }
                     // DIRECT blocks: every valid pair has rel index p(i) - p(j) = rbase + c
                     // within the table and no candidate row (lanes without a valid pair
                     // read the guarded table at base 0)
@@ -706,7 +749,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         idle || ((vb & candbits) == 0u && rb + c_lo >= 0 && rb + c_hi <= p.R - 1);
                     const bool direct =
                         !use_rel || (rel_in_smem && __all_sync(0xffffffffu, lane_direct));
-                    e.rbase = idle ? 0 : rb;
+                    e.rbase = (idle || !use_rel) ? 0 : rb;   // R = 0: all-zero guard band
                     e.tq32 = tsq32 + st * BM + wq * QW;
                     e.tq64 = tsq + st * BM + wq * QW;
                     HalfTime ht = {};
@@ -730,44 +773,42 @@ __global__ void __launch_bounds__(kThreads, 1)
                         else if (tmode == 2) epi_block<2, false>(p, e, ht, k, t_lo, t_hi);
                         else epi_block<3, false>(p, e, ht, k, t_lo, t_hi);
                     }
-                    tmem_wait_st();
-                    tc_fence_before();
-                    fence_proxy_async_smem();
-                    warp_arrive(&bars[P_FULL]);
-                    warp_arrive(&bars[EPI_DONE + st]);
                     if (use_ts && tmode == 1) {
                         run_add(k, tb_slot, ht.blo, t_lo);
                         run_add(k, tb_slot, ht.blo + 1, t_hi);
                     }
                     if (use_rel) flush_rel(p, k, e.iq, jw, e.Em1, hrel, args.d_rel, rel_in_smem);
                 }
+                tmem_wait_st();
+                tc_fence_before();
+                fence_proxy_async_smem();
+                warp_arrive(&bars[P_FULL]);
+                warp_arrive(&bars[EPI_DONE + st]);
 
                 // ---- dQ tile: lanes = query rows of this tile; columns split by warpgroup
                 if (!warp_wait(&bars[DQ_FULL], g & 1)) { ok = false; break; }
                 tc_fence_after();
                 {
-                    constexpr int QC = DQK / 4;
+                    constexpr int QC = DQK / kGroups;          // 16, 32 or 64 columns
                     const int i = t.qt * BM + r;
-                    uint32_t rq[32];
-                    if (QC == 32) {
-                        tmem_ld32(tl + kColDP + wq * QC, rq);
-                    } else {
-                        uint32_t (&r16)[16] = *reinterpret_cast<uint32_t(*)[16]>(rq);
-                        tmem_ld16(tl + kColDP + wq * QC, r16);
-                    }
-                    tmem_wait_ld();
-                    reg_fence(rq);
-                    tc_fence_before();
-                    warp_arrive(&bars[DQ_FREE]);
-                    if (i < s.L) {
-                        float *dqr = args.dq_acc + ((s.start + i) * (int64_t)p.H + un.h) * DQK + wq * QC;
+                    const bool row_in = i < s.L;
+                    float *dqr = args.dq_acc + ((s.start + i) * (int64_t)p.H + un.h) * DQK + wg * QC;
+                    const float al = p.alpha;
+                    tmem_row_foreach<QC>(tl + kColDP + wg * QC, [&](int c0, const auto &v) {
+                        constexpr int NV = sizeof(v) / sizeof(v[0]);
+                        if (c0 + NV >= QC) {                     // the last piece is in registers
+                            tc_fence_before();
+                            warp_arrive(&bars[DQ_FREE]);
+                        }
+                        if (row_in) {
 #pragma unroll
-                        for (int q = 0; q < QC / 4; ++q)
-                            red_add_v4(dqr + 4 * q, p.alpha * __uint_as_float(rq[4 * q]),
-                                       p.alpha * __uint_as_float(rq[4 * q + 1]),
-                                       p.alpha * __uint_as_float(rq[4 * q + 2]),
-                                       p.alpha * __uint_as_float(rq[4 * q + 3]));
-                    }
+                            for (int q = 0; q < NV / 4; ++q)
+                                red_add_v4(dqr + c0 + 4 * q, al * __uint_as_float(v[4 * q]),
+                                           al * __uint_as_float(v[4 * q + 1]),
+                                           al * __uint_as_float(v[4 * q + 2]),
+                                           al * __uint_as_float(v[4 * q + 3]));
+                        }
+                    });
                 }
                 ++x;
                 ++g;
@@ -778,45 +819,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!warp_wait(&bars[ACC_FULL], n & 1)) { ok = false; break; }
             tc_fence_after();
             {
-                constexpr int VC = DV / 4, KC = DQK / 4;
-                uint32_t ra[32], rk[32];
-                if (VC == 32) {
-                    tmem_ld32(tl + kColDV + wq * VC, ra);
-                } else {
-                    uint32_t (&r16)[16] = *reinterpret_cast<uint32_t(*)[16]>(ra);
-                    tmem_ld16(tl + kColDV + wq * VC, r16);
-                }
-                if (KC == 32) {
-                    tmem_ld32(tl + kColDK + wq * KC, rk);
-                } else {
-                    uint32_t (&r16)[16] = *reinterpret_cast<uint32_t(*)[16]>(rk);
-                    tmem_ld16(tl + kColDK + wq * KC, r16);
-                }
-                tmem_wait_ld();
-                reg_fence(ra);
-                reg_fence(rk);
+                constexpr int VC = DV / kGroups, KC = DQK / kGroups;
+                const int64_t row = (s.start + k.j) * (int64_t)p.H + un.h;
+                const float sv = x > 0 ? 1.0f : 0.f, sk = x > 0 ? p.alpha : 0.f;
+                __nv_bfloat16 *dvr = args.dv + row * DV + wg * VC;
+                __nv_bfloat16 *dkr = args.dk + row * DQK + wg * KC;
+                const bool key_in = k.key_in;
+                tmem_row_foreach<VC>(tl + kColDV + wg * VC, [&](int c0, const auto &v) {
+                    if (key_in) store_bf16_row(dvr + c0, v, sv);
+                });
+                tmem_row_foreach<KC>(tl + kColDK + wg * KC, [&](int c0, const auto &v) {
+                    if (key_in) store_bf16_row(dkr + c0, v, sk);
+                });
                 tc_fence_before();
                 warp_arrive(&bars[ACC_FREE]);
-                if (k.key_in) {
-                    const int64_t row = (s.start + k.j) * (int64_t)p.H + un.h;
-                    const float sv = x > 0 ? 1.0f : 0.f, sk = x > 0 ? p.alpha : 0.f;
-                    uint4 *dvp = reinterpret_cast<uint4 *>(args.dv + row * DV + wq * VC);
-                    uint4 *dkp = reinterpret_cast<uint4 *>(args.dk + row * DQK + wq * KC);
-#pragma unroll
-                    for (int q = 0; q < VC / 8; ++q)
-                        dvp[q] = make_uint4(
-                            pack_bf16x2(sv * __uint_as_float(ra[8 * q]), sv * __uint_as_float(ra[8 * q + 1])),
-                            pack_bf16x2(sv * __uint_as_float(ra[8 * q + 2]), sv * __uint_as_float(ra[8 * q + 3])),
-                            pack_bf16x2(sv * __uint_as_float(ra[8 * q + 4]), sv * __uint_as_float(ra[8 * q + 5])),
-                            pack_bf16x2(sv * __uint_as_float(ra[8 * q + 6]), sv * __uint_as_float(ra[8 * q + 7])));
-#pragma unroll
-                    for (int q = 0; q < KC / 8; ++q)
-                        dkp[q] = make_uint4(
-                            pack_bf16x2(sk * __uint_as_float(rk[8 * q]), sk * __uint_as_float(rk[8 * q + 1])),
-                            pack_bf16x2(sk * __uint_as_float(rk[8 * q + 2]), sk * __uint_as_float(rk[8 * q + 3])),
-                            pack_bf16x2(sk * __uint_as_float(rk[8 * q + 4]), sk * __uint_as_float(rk[8 * q + 5])),
-                            pack_bf16x2(sk * __uint_as_float(rk[8 * q + 6]), sk * __uint_as_float(rk[8 * q + 7])));
-                }
             }
             ++n;
         }
@@ -824,7 +840,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     tc_fence_before();
-    __threadfence();   // reductions into the slot row are complete before it is read back
+    fence_gpu();   // reductions into the slot row are complete before it is read back
     __syncthreads();
     // fold this CTA's table-gradient histograms into the outputs
     if (rel_in_smem)
