@@ -21,6 +21,15 @@ template <typename T>
 cudaError_t launch_ln_gate_bwd(const DevParams &p, const void *dout, const void *u,
                                const float *y, const float *mean, const float *rstd, void *du,
                                void *dy, bool dy_bf16, cudaStream_t st);
+// Vectorised LayerNorm + gating (norm.cu) for rows of 128*k features (k <= 8 or 16).
+bool ln_vec_supported(int D);
+template <typename T>
+cudaError_t launch_ln_gate_vec(const DevParams &p, const float *y, const void *u, void *out,
+                               float *mean, float *rstd, cudaStream_t st);
+template <typename T>
+cudaError_t launch_ln_gate_bwd_vec(const DevParams &p, const void *dout, const void *u,
+                                   const float *y, const float *mean, const float *rstd,
+                                   void *du, void *dy, bool dy_bf16, cudaStream_t st);
 template <typename T>
 cudaError_t launch_simt_bwd(const DevParams &p, const void *q, const void *k, const void *v,
                             const float *dy, float *dq_acc, void *dk, void *dv, float *d_rel,

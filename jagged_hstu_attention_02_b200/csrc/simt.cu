@@ -497,6 +497,7 @@ template <typename T>
 cudaError_t launch_ln_gate(const DevParams &p, const float *y, const void *u, void *out,
                            float *mean, float *rstd, cudaStream_t st)
 {
+    if (ln_vec_supported(p.D)) return launch_ln_gate_vec<T>(p, y, u, out, mean, rstd, st);
     const int rows_per_block = kThreads / 32;
     const int64_t blocks = (p.T + rows_per_block - 1) / rows_per_block;
     ln_gate_kernel<T><<<(unsigned)blocks, kThreads, 0, st>>>(p, y, (const T *)u, (T *)out, mean,
@@ -509,6 +510,8 @@ cudaError_t launch_ln_gate_bwd(const DevParams &p, const void *dout, const void 
                                const float *y, const float *mean, const float *rstd, void *du,
                                void *dy, bool dy_bf16, cudaStream_t st)
 {
+    if (ln_vec_supported(p.D))
+        return launch_ln_gate_bwd_vec<T>(p, dout, u, y, mean, rstd, du, dy, dy_bf16, st);
     const int rows_per_block = kThreads / 32;
     const int64_t blocks = (p.T + rows_per_block - 1) / rows_per_block;
     if (dy_bf16)
