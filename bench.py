@@ -169,7 +169,13 @@ def run_ours(args, world, rank, local):
     dev = ops.batch_to_device(b)
     kw = ops.batch_kwargs(b)
     out, saved = ops.run_fwd(b, dev, training=True)
-    grads = ops.run_bwd(b, saved, dev_tensors=dev)
+    # the bias-table gradients live in one buffer: a sharded step sums them across ranks
+    # with one all-reduce (jagged_hstu_attention_02_b200.shard), the only exchange it has
+    R, NB = b.rel_bias_len, b.time_bias_len
+    table_grads = torch.zeros(R + NB, dtype=torch.float32, device="cuda")
+    grads = (torch.empty_like(dev["q"]), torch.empty_like(dev["k"]), torch.empty_like(dev["v"]),
+             torch.empty_like(dev["u"]), table_grads[:R], table_grads[R:])
+    ops.run_bwd(b, saved, dev_tensors=dev, grads=grads)
     ws_f = ops.fwd.last_workspace
     ws_b = ops.bwd.last_workspace
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
@@ -181,6 +187,8 @@ def run_ours(args, world, rank, local):
         ops.bwd(dev["dout"], dev["q"], dev["k"], dev["v"], dev["u"], dev["seq_offsets"],
                 dev["num_contextuals"], dev["num_targets"], dev["timestamps"], dev["rel_bias"],
                 dev["time_bias"], saved=saved, grads=grads, workspace=ws_b, **kw)
+        if world > 1:
+            torch.distributed.all_reduce(table_grads)
 
     stages = ["fwd_attn", "fwd_norm", "bwd_norm", "bwd_attn"]
     for _ in range(args.warmup):
