@@ -128,6 +128,7 @@ struct UnitIter {
             const int rem = (int)(u % bh);
             b = rem / p.H;
             h = rem % p.H;
+            if (!seq_may_have_tile(p, b, kt)) continue;
             s = load_seq(p, b, report && kt == 0 && h == 0);
             if (kt * BN < s.L) return true;
         }
@@ -486,6 +487,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             rels[p.R + x] = 0.f;
         }
     }
+    fill_seq_tiles(p, kThreads);
     __threadfence();   // the zeroed slot row is in place before any reduction into it
     __syncthreads();
     if (p.NB > 0) build_lut(thr, p.n_thr, lut, lut_valid);
@@ -791,7 +793,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 {
                     constexpr int QC = DQK / kGroups;          // 16, 32 or 64 columns
                     const int i = t.qt * BM + r;
-                    const bool row_in = i < s.L;
                     float *dqr = args.dq_acc + ((s.start + i) * (int64_t)p.H + un.h) * DQK + wg * QC;
                     const float al = p.alpha;
                     tmem_row_foreach<QC>(tl + kColDP + wg * QC, [&](int c0, const auto &v) {
@@ -800,14 +801,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                             tc_fence_before();
                             warp_arrive(&bars[DQ_FREE]);
                         }
-                        if (row_in) {
+                        // the NV/4 lanes of a group add one row's chunks side by side
+                        constexpr int NCH = NV / 4;
+                        float4 xc[NCH];
 #pragma unroll
-                            for (int q = 0; q < NV / 4; ++q)
-                                red_add_v4(dqr + c0 + 4 * q, al * __uint_as_float(v[4 * q]),
-                                           al * __uint_as_float(v[4 * q + 1]),
-                                           al * __uint_as_float(v[4 * q + 2]),
-                                           al * __uint_as_float(v[4 * q + 3]));
-                        }
+                        for (int q = 0; q < NCH; ++q)
+                            xc[q] = make_float4(al * __uint_as_float(v[4 * q]),
+                                                al * __uint_as_float(v[4 * q + 1]),
+                                                al * __uint_as_float(v[4 * q + 2]),
+                                                al * __uint_as_float(v[4 * q + 3]));
+                        transpose_chunks<NCH>(xc);
+                        const int jl = lane % NCH, r0 = i - jl;   // rows r0 .. r0 + NCH - 1
+                        float *dqb = dqr - (int64_t)jl * p.H * DQK + c0 + 4 * jl;
+#pragma unroll
+                        for (int c = 0; c < NCH; ++c)
+                            if (r0 + c < s.L)
+                                red_add_v4(dqb + (int64_t)c * p.H * DQK, xc[c].x, xc[c].y,
+                                           xc[c].z, xc[c].w);
                     });
                 }
                 ++x;
@@ -860,7 +870,8 @@ template <int DQK, int DV>
 cudaError_t launch_bwd(const BwdTcArgs &a, cudaStream_t st)
 {
     using L = BwdLayout<DQK, DV>;
-    static_assert(L::ALLOC <= 232448, "shared memory layout exceeds the per-CTA limit");
+    static_assert(L::ALLOC + kSeqTileCache <= 232448,
+                  "shared memory layout exceeds the per-CTA limit");
     auto kern = bwd_tc_kernel<DQK, DV>;
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);

@@ -70,6 +70,57 @@ __device__ __forceinline__ SeqInfo load_seq(const DevParams &p, int b, bool repo
     return s;
 }
 
+// Tiles of 128 rows of each sequence (ceil(L/128), saturated at 255; 0 for an invalid
+// sequence, which is reported here), cached in shared memory by the persistent kernels so
+// that their work-unit iterators step over units past a sequence's end without a chain of
+// global loads.  A static array: its address is a constant, so the iterators keep no
+// pointer to it.  Batches of more than kSeqTileCache sequences skip the cache.
+constexpr int kSeqTileCache = 3072;
+static __shared__ uint8_t s_seq_tiles[kSeqTileCache];
+
+__device__ __forceinline__ void fill_seq_tiles(const DevParams &p, int nthreads)
+{
+    if (p.B > kSeqTileCache) return;
+    for (int b = threadIdx.x; b < p.B; b += nthreads) {
+        const SeqInfo s = load_seq(p, b, true);
+        s_seq_tiles[b] = (uint8_t)min((s.L + 127) / 128, 255);
+    }
+}
+
+// False only when the cache shows that sequence b has no tile t.
+__device__ __forceinline__ bool seq_may_have_tile(const DevParams &p, int b, int t)
+{
+    if (p.B > kSeqTileCache) return true;
+    const int n = s_seq_tiles[b];
+    return t < n || n == 255;
+}
+
+// Transposes 16-byte chunks within groups of NCH lanes: on entry lane l holds chunks
+// 0..NCH-1 of row l; on exit lane l, j = l % NCH, holds chunk j of rows l - j .. l - j +
+// NCH-1 (slot c = row l - j + c).  Lets the NCH lanes of a group write one row's NCH
+// chunks side by side (whole 128-byte lines for NCH = 8) instead of each lane writing its
+// own row.  Butterfly of xor shuffles, log2(NCH) rounds.
+template <int NCH>
+__device__ __forceinline__ void transpose_chunks(float4 (&x)[NCH])
+{
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int m = NCH / 2; m >= 1; m >>= 1) {
+        const bool hi = (lane & m) != 0;
+#pragma unroll
+        for (int c = 0; c < NCH; ++c) {
+            if (c & m) continue;
+            const float4 snd = hi ? x[c] : x[c | m];
+            float4 rcv;
+            rcv.x = __shfl_xor_sync(0xffffffffu, snd.x, m);
+            rcv.y = __shfl_xor_sync(0xffffffffu, snd.y, m);
+            rcv.z = __shfl_xor_sync(0xffffffffu, snd.z, m);
+            rcv.w = __shfl_xor_sync(0xffffffffu, snd.w, m);
+            if (hi) x[c] = rcv; else x[c | m] = rcv;
+        }
+    }
+}
+
 // p(x): candidates take the last history position.
 __device__ __forceinline__ int clamp_pos(int x, int E) { return (E > 0 && x >= E) ? E - 1 : x; }
 

@@ -95,12 +95,19 @@ struct FwdTcArgs {
 // Visits the key tiles of query tile [i0, i0+BM) that hold a valid pair, in order.
 struct TileIter {
     const SeqInfo &s;
-    int i0, W, kt, nkt;
+    int i0, W, kt;
+    // Valid pairs have j <= i, except contextual rows, which see the whole contextual
+    // prefix: the first candidate key tile is the later of the diagonal and the prefix's end.
     __device__ TileIter(const SeqInfo &s_, int i0_, int W_)
-        : s(s_), i0(i0_), W(W_), kt(-1), nkt((s_.L + BN - 1) / BN) {}
+        : s(s_), i0(i0_), W(W_),
+          kt(min((s_.L + BN - 1) / BN, max(i0_ / BN, (s_.c - 1) / BN) + 1)) {}
+    // Descending: the diagonal tile, the most expensive one of a unit (masks, clamped
+    // positions, many time buckets), comes first, where the double-buffered S and A absorb
+    // the spread between warps, instead of last, where every warp would wait for the
+    // slowest one before the unit's output can be read.
     __device__ bool next()
     {
-        while (++kt < nkt)
+        while (--kt >= 0)
             if (tile_any_valid(i0, i0 + BM - 1, kt * BN, kt * BN + BN - 1, s, W)) return true;
         return false;
     }
@@ -127,6 +134,7 @@ struct UnitIter {
             const int rem = (int)(u % bh);
             b = rem / p.H;
             h = rem % p.H;
+            if (!seq_may_have_tile(p, b, qt)) continue;
             s = load_seq(p, b, report && qt == 0 && h == 0);
             if (qt * BM < s.L) return true;
         }
@@ -201,6 +209,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const bool rel_in_smem = p.R <= kRelSmemMax;
     if (rel_in_smem)
         for (int x = threadIdx.x; x < p.R; x += kTcThreads) relh[x] = tscale * p.rel[x];
+    fill_seq_tiles(p, kTcThreads);
     __syncthreads();
     if (p.NB > 0) build_lut(thr, p.n_thr, lutp, lut_valid);
     tc_fence_before();
@@ -464,6 +473,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 // ---- per (row, quarter tile) structure; path choices are made warp-uniform
                 const uint32_t vmask = full ? 0xFFFFFFFFu : (uint32_t)row_valid_bits(i, jq, s, p.W);
                 const int rbase = pi - jq;            // rel index of key jq + c is rbase - c
+                // a 32 x 32 block without a valid pair only writes zeros into A
+                const bool blk_any = __any_sync(0xffffffffu, vmask != 0u);
                 const bool rdirect =
                     __all_sync(0xffffffffu, !use_rel || (rbase - (QW - 1) >= 0 && rbase <= p.R - 1));
                 HalfTime ht = {};
@@ -481,6 +492,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     break;
                 }
                 tc_fence_after();
+                if (!blk_any) {
+                    // this quarter's A columns (SPLIT: hi and lo parts, 32 columns)
+                    if constexpr (SPLIT) {
+                        tmem_zero16(tmem + lane_base + kPCol + wq * 32);
+                        tmem_zero16(tmem + lane_base + kPCol + wq * 32 + 16);
+                    } else {
+                        tmem_zero16(tmem + lane_base + kPCol + ps * 64 + wq * 16);
+                    }
+                } else {
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
                     const int cb = hf * 16;
@@ -564,6 +584,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         tmem_st8(tmem + lane_base + kPCol + ps * 64 + wq * 16 + hf * 8, pk);
                     }
                 }
+                }
                 tmem_wait_st();
                 tc_fence_before();
                 warp_arrive(&bars[P_FULL + ps]);
@@ -575,7 +596,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             if (!warp_wait(&bars[O_FULL], n & 1)) { ok = false; break; }
             tc_fence_after();
             constexpr int OC = DV / 4;                // 32 or 16 output columns per warpgroup
-            float *yr = args.y + (s.start + i) * (int64_t)p.D + un.h * DV + wq * OC;
             uint32_t ro[32];
             if (OC == 32) {
                 tmem_ld32(tmem + lane_base + kOCol + wq * OC, ro);
@@ -587,14 +607,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             reg_fence(ro);
             tc_fence_before();
             warp_arrive(&bars[O_FREE]);
-            if (row_in) {
-                float4 *dst = reinterpret_cast<float4 *>(yr);
+            {
+                // lanes of a group of OC/4 write one row's chunks side by side
+                constexpr int NCH = OC / 4;
+                float4 yc[NCH];
 #pragma unroll
-                for (int x = 0; x < OC / 4; ++x)
-                    dst[x] = make_float4(__uint_as_float(ro[4 * x]) * p.inv_N,
-                                         __uint_as_float(ro[4 * x + 1]) * p.inv_N,
-                                         __uint_as_float(ro[4 * x + 2]) * p.inv_N,
-                                         __uint_as_float(ro[4 * x + 3]) * p.inv_N);
+                for (int x = 0; x < NCH; ++x)
+                    yc[x] = make_float4(__uint_as_float(ro[4 * x]) * p.inv_N,
+                                        __uint_as_float(ro[4 * x + 1]) * p.inv_N,
+                                        __uint_as_float(ro[4 * x + 2]) * p.inv_N,
+                                        __uint_as_float(ro[4 * x + 3]) * p.inv_N);
+                transpose_chunks<NCH>(yc);
+                const int j = lane % NCH, r0 = i - j;         // rows r0 .. r0 + NCH - 1
+                float *yb = args.y + (s.start + r0) * (int64_t)p.D + un.h * DV + wq * OC + 4 * j;
+#pragma unroll
+                for (int c = 0; c < NCH; ++c)
+                    if (r0 + c < s.L)
+                        *reinterpret_cast<float4 *>(yb + (int64_t)c * p.D) = yc[c];
             }
             ++n;
         }
@@ -632,7 +661,8 @@ template <int DQK, int DV>
 cudaError_t launch_tc(const FwdTcArgs &a, bool split, cudaStream_t st)
 {
     using L = FwdLayout<DQK, DV>;
-    static_assert(L::ALLOC <= 232448, "shared memory layout exceeds the per-CTA limit");
+    static_assert(L::ALLOC + kSeqTileCache <= 232448,
+                  "shared memory layout exceeds the per-CTA limit");
     auto kern = split ? fwd_tc_kernel<DQK, DV, true> : fwd_tc_kernel<DQK, DV, false>;
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);

@@ -257,6 +257,17 @@ __device__ __forceinline__ void tmem_st4(uint32_t taddr, const uint32_t (&r)[4])
                  : "memory");
 }
 
+// Zeroes 16 consecutive 32-bit columns of this thread's TMEM lane (one source register).
+__device__ __forceinline__ void tmem_zero16(uint32_t taddr)
+{
+    const uint32_t z = 0u;
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1};" ::"r"(taddr),
+        "r"(z)
+        : "memory");
+}
+
 // Stores 8 consecutive 32-bit columns of this thread's TMEM lane.
 __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8])
 {
