@@ -75,7 +75,7 @@ __device__ __forceinline__ SeqInfo load_seq(const DevParams &p, int b, bool repo
 // that their work-unit iterators step over units past a sequence's end without a chain of
 // global loads.  A static array: its address is a constant, so the iterators keep no
 // pointer to it.  Batches of more than kSeqTileCache sequences skip the cache.
-constexpr int kSeqTileCache = 3072;
+constexpr int kSeqTileCache = 2048;
 static __shared__ uint8_t s_seq_tiles[kSeqTileCache];
 
 __device__ __forceinline__ void fill_seq_tiles(const DevParams &p, int nthreads)

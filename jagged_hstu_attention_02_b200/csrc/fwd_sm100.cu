@@ -46,7 +46,7 @@ namespace {
 constexpr int BM = 128, BN = 128, QW = 32;   // QW: key columns per epilogue warpgroup
 constexpr int kEpiWarps = 16;                  // four warpgroups
 constexpr int kTcThreads = 128 + 32 * kEpiWarps;
-constexpr int kRelSmemMax = 4096;
+constexpr int kRelSmemMax = 4352;   // covers N up to 4351 (R = N + 1)
 constexpr uint32_t kTmemCols = 512;
 constexpr int kBlockBytes = 128 * 128;   // one 128-row x 64-element bf16 swizzle block
 constexpr uint32_t kPCol = 256;          // TMEM columns of A (packed bf16)
@@ -164,6 +164,107 @@ __device__ __forceinline__ void warp_arrive(uint64_t *bar)
 // LayerNorm gradient is sensitive to the error of Y).  Without SPLIT, A has two TMEM
 // buffers of 64 columns; with SPLIT one buffer of 128 (per 32-key quarter w: hi at
 // 32w..32w+15, lo at 32w+16..32w+31).
+// One 32-row x 32-key block of the epilogue (thread = row = TMEM lane): the bias, SiLU, the
+// mask, and A into TMEM.  The mode choices are template parameters, so the body has no
+// branch and the compiler can overlap the loads and arithmetic of neighbouring keys:
+//   TM   time bias: 0 one bucket, 1 one boundary, 2 lookup table, 3 64-bit search
+//   RD   rel index rbase - c without clamping
+//   FULL every pair of the block is valid (no mask)
+struct FwdEpi {
+    uint32_t t_s;              // TMEM address of the block's S columns
+    uint32_t t_a;              // TMEM address of the block's A columns
+    const int32_t *tk32;       // key stamps relative to the quarter's minimum
+    const int64_t *tk64;       // and absolute
+    const float *relp;         // rel table (relp * rel_sc = half bias)
+    float rel_sc;
+    int rbase, R;              // rel index of key c: rbase - c (clamped unless RD)
+    float half_alpha, alpha;
+    const float *tbh;          // half time-bias table
+    const LutEntry *lut;
+    const uint64_t *thr;
+    int n_thr;
+    int64_t tsi;               // the row's stamp
+};
+
+template <int TM, bool RD, bool FULL, bool SPLIT>
+__device__ __forceinline__ void fwd_quarter(const FwdEpi &e, const HalfTime &ht, uint32_t vmask)
+{
+    // one-boundary test as a single unsigned compare: the key is in the lower bucket when
+    // cmpA < t < cmpB
+    const uint32_t a1 = (uint32_t)ht.cmpA + 1u;
+    const int64_t sp = (int64_t)ht.cmpB - (int64_t)ht.cmpA - 1;
+    const uint32_t span = sp > 0 ? (uint32_t)sp : 0u;
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+        const int cb = hf * 16;
+        uint32_t ra[16];
+        tmem_ld16(e.t_s + cb, ra);
+        tmem_wait_ld();
+        reg_fence(ra);
+        float bh[16];   // half of the bias
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+            float tb;
+            if (TM == 0) {
+                tb = ht.tb_lo;
+            } else if (TM == 1) {
+                const bool lo = (uint32_t)e.tk32[cb + c] - a1 < span;
+                tb = lo ? ht.tb_lo : ht.tb_hi;
+            } else if (TM == 2) {
+                const int32_t d = ht.t_rel - e.tk32[cb + c];
+                uint32_t dt = (uint32_t)(d < 0 ? -d : d);
+                dt = min(dt, (uint32_t)INT32_MAX - 1u);
+                const float v = e.tbh[lut_bucket(e.lut, dt)];
+                tb = ht.lane_const ? ht.tb_lo : v;
+            } else {
+                tb = e.tbh[bucket_search(e.thr, e.n_thr, abs_diff_u64(e.tsi, e.tk64[cb + c]))];
+            }
+            int ri = e.rbase - cb - c;
+            if (!RD) ri = ri < 0 ? 0 : (ri > e.R - 1 ? e.R - 1 : ri);
+            bh[c] = fmaf(e.relp[ri], e.rel_sc, tb);
+        }
+        // SiLU(x) = x sigmoid(x) = h + h tanh(h), h = x/2; mask after the nonlinearity
+        const uint32_t vb = vmask >> cb;
+        uint32_t pk[8];
+        if constexpr (SPLIT) {
+            // training forward: accurate sigmoid in fp32, A split into hi + lo
+            uint32_t plo[8];
+#pragma unroll
+            for (int c2 = 0; c2 < 8; ++c2) {
+                float a[2];
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    const int c = 2 * c2 + q;
+                    const float xs = fmaf(e.alpha, __uint_as_float(ra[c]), 2.0f * bh[c]);
+                    const float v = xs * __fdividef(1.0f, 1.0f + __expf(-xs));
+                    a[q] = (FULL || ((vb >> c) & 1u)) ? v : 0.f;
+                }
+                pk[c2] = pack_bf16x2(a[0], a[1]);
+                plo[c2] = pack_bf16x2(a[0] - __uint_as_float(pk[c2] << 16),
+                                      a[1] - __uint_as_float(pk[c2] & 0xFFFF0000u));
+            }
+            tmem_st8(e.t_a + hf * 8, pk);
+            tmem_st8(e.t_a + 16 + hf * 8, plo);
+        } else {
+            // inference forward: h in fp32, then tanh and h + h tanh(h) on bf16 pairs
+            // (A is rounded to bf16 for the tensor core either way)
+#pragma unroll
+            for (int c2 = 0; c2 < 8; ++c2) {
+                const float x0 = fmaf(e.half_alpha, __uint_as_float(ra[2 * c2]), bh[2 * c2]);
+                const float x1 = fmaf(e.half_alpha, __uint_as_float(ra[2 * c2 + 1]), bh[2 * c2 + 1]);
+                // bf16 pair = the high halves of x0, x1 (one byte permute)
+                const uint32_t h2 = __byte_perm(__float_as_uint(x0), __float_as_uint(x1), 0x7632);
+                uint32_t a2 = fma_bf16x2(h2, tanh_bf16x2(h2), h2);
+                if (!FULL)
+                    a2 &= (((vb >> (2 * c2)) & 1u) ? 0x0000FFFFu : 0u) |
+                          (((vb >> (2 * c2 + 1)) & 1u) ? 0xFFFF0000u : 0u);
+                pk[c2] = a2;
+            }
+            tmem_st8(e.t_a + hf * 8, pk);
+        }
+    }
+}
+
 template <int DQK, int DV, bool SPLIT>
 __global__ void __launch_bounds__(kTcThreads, 1)
     fwd_tc_kernel(const __grid_constant__ FwdTcArgs args)
@@ -209,6 +310,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const bool rel_in_smem = p.R <= kRelSmemMax;
     if (rel_in_smem)
         for (int x = threadIdx.x; x < p.R; x += kTcThreads) relh[x] = tscale * p.rel[x];
+    if (p.R == 0 && threadIdx.x == 0) relh[0] = 0.f;   // read, times zero bias, without a table
     fill_seq_tiles(p, kTcThreads);
     __syncthreads();
     if (p.NB > 0) build_lut(thr, p.n_thr, lutp, lut_valid);
@@ -462,21 +564,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     ok = false;
                     break;
                 }
-                tc_fence_after();
-                uint32_t ra[32];
-                tmem_ld32(tmem + lane_base + st * 128 + wq * QW, ra);
-                tmem_wait_ld();
-                reg_fence(ra);
-                tc_fence_before();
-                warp_arrive(&bars[S_FREE + st]);      // S is in registers: release it
-
                 // ---- per (row, quarter tile) structure; path choices are made warp-uniform
                 const uint32_t vmask = full ? 0xFFFFFFFFu : (uint32_t)row_valid_bits(i, jq, s, p.W);
                 const int rbase = pi - jq;            // rel index of key jq + c is rbase - c
                 // a 32 x 32 block without a valid pair only writes zeros into A
                 const bool blk_any = __any_sync(0xffffffffu, vmask != 0u);
+                // without a rel table the clamped path reads the single zero entry
                 const bool rdirect =
-                    __all_sync(0xffffffffu, !use_rel || (rbase - (QW - 1) >= 0 && rbase <= p.R - 1));
+                    use_rel && __all_sync(0xffffffffu, rbase - (QW - 1) >= 0 && rbase <= p.R - 1);
                 HalfTime ht = {};
                 int tmode = 0;
                 if (use_ts) {
@@ -484,8 +579,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                                          meta[st].tmax[wq], meta[st].ok32[wq] != 0, lut_ok, lutp);
                     tmode = __reduce_max_sync(0xffffffffu, ht.my_mode);
                 }
-                const int32_t *tk32 = tsk32 + st * BN + wq * QW;
-                const int64_t *tk64 = tsk + st * BN + wq * QW;
+                FwdEpi e;
+                e.t_s = tmem + lane_base + st * 128 + wq * QW;
+                e.t_a = SPLIT ? tmem + lane_base + kPCol + wq * 32
+                              : tmem + lane_base + kPCol + ps * 64 + wq * 16;
+                e.tk32 = tsk32 + st * BN + wq * QW;
+                e.tk64 = tsk + st * BN + wq * QW;
+                e.relp = use_rel ? relp : relh;
+                e.rel_sc = rel_sc;
+                e.rbase = use_rel ? rbase : 0;
+                e.R = use_rel ? p.R : 1;
+                e.half_alpha = half_alpha;
+                e.alpha = p.alpha;
+                e.tbh = tbh;
+                e.lut = lutp;
+                e.thr = thr;
+                e.n_thr = p.n_thr;
+                e.tsi = tsi;
                 // A's buffer is free once the A V of tile g - NP has completed
                 if (g >= NP && !warp_wait(&bars[P_FREE + ps], ((g / NP) - 1) & 1)) {
                     ok = false;
@@ -494,97 +604,25 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 tc_fence_after();
                 if (!blk_any) {
                     // this quarter's A columns (SPLIT: hi and lo parts, 32 columns)
-                    if constexpr (SPLIT) {
-                        tmem_zero16(tmem + lane_base + kPCol + wq * 32);
-                        tmem_zero16(tmem + lane_base + kPCol + wq * 32 + 16);
-                    } else {
-                        tmem_zero16(tmem + lane_base + kPCol + ps * 64 + wq * 16);
-                    }
+                    tmem_zero16(e.t_a);
+                    if constexpr (SPLIT) tmem_zero16(e.t_a + 16);
+                } else if (tmode == 3) {
+                    fwd_quarter<3, false, false, SPLIT>(e, ht, vmask);
+                } else if (full && rdirect) {
+                    if (tmode == 0) fwd_quarter<0, true, true, SPLIT>(e, ht, vmask);
+                    else if (tmode == 1) fwd_quarter<1, true, true, SPLIT>(e, ht, vmask);
+                    else fwd_quarter<2, true, true, SPLIT>(e, ht, vmask);
+                } else if (rdirect) {
+                    if (tmode == 0) fwd_quarter<0, true, false, SPLIT>(e, ht, vmask);
+                    else if (tmode == 1) fwd_quarter<1, true, false, SPLIT>(e, ht, vmask);
+                    else fwd_quarter<2, true, false, SPLIT>(e, ht, vmask);
                 } else {
-#pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
-                    const int cb = hf * 16;
-                    float bh[16];   // scaled half of the bias, time part first
-                    if (tmode == 0) {
-#pragma unroll
-                        for (int c = 0; c < 16; ++c) bh[c] = ht.tb_lo;
-                    } else if (tmode == 1) {
-#pragma unroll
-                        for (int c = 0; c < 16; ++c) {
-                            const int32_t tj = tk32[cb + c];
-                            bh[c] = (tj <= ht.cmpA || tj >= ht.cmpB) ? ht.tb_hi : ht.tb_lo;
-                        }
-                    } else if (tmode == 2) {
-#pragma unroll
-                        for (int c = 0; c < 16; ++c) {
-                            int32_t d = ht.t_rel - tk32[cb + c];
-                            uint32_t dt = (uint32_t)(d < 0 ? -d : d);
-                            dt = min(dt, (uint32_t)INT32_MAX - 1u);
-                            const float v = tbh[lut_bucket(lutp, dt)];
-                            bh[c] = ht.lane_const ? ht.tb_lo : v;
-                        }
-                    } else {
-#pragma unroll
-                        for (int c = 0; c < 16; ++c)
-                            bh[c] = tbh[bucket_search(thr, p.n_thr, abs_diff_u64(tsi, tk64[cb + c]))];
-                    }
-                    if (use_rel) {
-                        if (rdirect) {
-                            const float *rr = relp + (rbase - cb);
-#pragma unroll
-                            for (int c = 0; c < 16; ++c) bh[c] = fmaf(rr[-c], rel_sc, bh[c]);
-                        } else {
-#pragma unroll
-                            for (int c = 0; c < 16; ++c) {
-                                int ri = rbase - cb - c;
-                                ri = ri < 0 ? 0 : (ri > p.R - 1 ? p.R - 1 : ri);
-                                bh[c] = fmaf(relp[ri], rel_sc, bh[c]);
-                            }
-                        }
-                    }
-                    // SiLU(x) = x sigmoid(x) = h + h tanh(h), h = x/2; mask after the nonlinearity
-                    uint32_t pk[8];
-                    const uint32_t vb = vmask >> cb;
-                    if constexpr (SPLIT) {
-                        // training forward: accurate sigmoid in fp32, A split into hi + lo
-                        uint32_t plo[8];
-#pragma unroll
-                        for (int c2 = 0; c2 < 8; ++c2) {
-                            float a[2];
-#pragma unroll
-                            for (int e = 0; e < 2; ++e) {
-                                const int c = 2 * c2 + e;
-                                const float xs = fmaf(p.alpha, __uint_as_float(ra[cb + c]), 2.0f * bh[c]);
-                                const float v = xs * __fdividef(1.0f, 1.0f + __expf(-xs));
-                                a[e] = full ? v : (((vb >> c) & 1u) ? v : 0.f);
-                            }
-                            pk[c2] = pack_bf16x2(a[0], a[1]);
-                            plo[c2] = pack_bf16x2(a[0] - __uint_as_float(pk[c2] << 16),
-                                                  a[1] - __uint_as_float(pk[c2] & 0xFFFF0000u));
-                        }
-                        tmem_st8(tmem + lane_base + kPCol + wq * 32 + hf * 8, pk);
-                        tmem_st8(tmem + lane_base + kPCol + wq * 32 + 16 + hf * 8, plo);
-                    } else {
-                        // inference forward: h in fp32, then tanh and h + h tanh(h) on bf16 pairs
-                        // (A is rounded to bf16 for the tensor core either way)
-#pragma unroll
-                        for (int c2 = 0; c2 < 8; ++c2) {
-                            const float x0 = fmaf(half_alpha, __uint_as_float(ra[cb + 2 * c2]), bh[2 * c2]);
-                            const float x1 =
-                                fmaf(half_alpha, __uint_as_float(ra[cb + 2 * c2 + 1]), bh[2 * c2 + 1]);
-                            // bf16 pair = the high halves of x0, x1 (one byte permute)
-                            const uint32_t h2 =
-                                __byte_perm(__float_as_uint(x0), __float_as_uint(x1), 0x7632);
-                            uint32_t a2 = fma_bf16x2(h2, tanh_bf16x2(h2), h2);
-                            if (!full)
-                                a2 &= (((vb >> (2 * c2)) & 1u) ? 0x0000FFFFu : 0u) |
-                                      (((vb >> (2 * c2 + 1)) & 1u) ? 0xFFFF0000u : 0u);
-                            pk[c2] = a2;
-                        }
-                        tmem_st8(tmem + lane_base + kPCol + ps * 64 + wq * 16 + hf * 8, pk);
-                    }
+                    if (tmode == 0) fwd_quarter<0, false, false, SPLIT>(e, ht, vmask);
+                    else if (tmode == 1) fwd_quarter<1, false, false, SPLIT>(e, ht, vmask);
+                    else fwd_quarter<2, false, false, SPLIT>(e, ht, vmask);
                 }
-                }
+                tc_fence_before();
+                warp_arrive(&bars[S_FREE + st]);      // S has been read
                 tmem_wait_st();
                 tc_fence_before();
                 warp_arrive(&bars[P_FULL + ps]);
