@@ -233,7 +233,8 @@ struct EpiBlock {
     uint32_t ds_row;              // smem address of this key's dS^T row (first 16-byte chunk)
     int ds_chunk0, rsw;           // first chunk of the block in the row, swizzle (row & 7)
     int iq;                       // first query of the block
-    int rbase;                    // p(iq) - p(j) in DIRECT blocks
+    int rbase;                    // p(iq) - p(j) in direct blocks (history columns)
+    int fc, rc;                   // first candidate column; this key's rel index for it
     int Em1;                      // p(i) = min(i, Em1)
     bool full, use_rel, use_ts, rel_in_smem;
     uint32_t vbits;               // valid queries of this key (bit c <-> query iq + c)
@@ -246,10 +247,14 @@ struct EpiBlock {
     float *tb_slot;
 };
 
-// DIRECT: every valid pair of the block has rel index p(i) - p(j) = rbase + c in [0, R)
-// (no candidate row, no clamping), and the table sits in shared memory with a guard band
-// that keeps the reads of masked pairs (at most 31 entries off) in bounds.
-template <int TM, bool DIRECT>
+// Rel index of a pair, by KIND:
+//   0  direct: every valid pair has index p(i) - p(j) = rbase + c in [0, R) (no candidate
+//      row, no clamping); the table sits in shared memory with a guard band that keeps the
+//      reads of masked pairs (at most 31 entries off) in bounds;
+//   1  direct for the history columns, and the candidate columns (c >= fc, p(i) = E - 1)
+//      at the lane's constant index rc;
+//   2  every index clamped, candidate / negative / out-of-table pairs sorted out per pair.
+template <int TM, int KIND>
 __device__ __forceinline__ void epi_block(const DevParams &p, const EpiBlock &e,
                                           const HalfTime &ht, KeyLane &k, float &t_lo,
                                           float &t_hi)
@@ -276,6 +281,8 @@ __device__ __forceinline__ void epi_block(const DevParams &p, const EpiBlock &e,
         reg_fence(rs);
         reg_fence(rd);
         uint32_t pa[4], pd[4];
+        int tbk[8];        // TM >= 2: bucket of each pair (-1: masked) and its dS
+        float tds[8];
 #pragma unroll
         for (int c2 = 0; c2 < 4; ++c2) {
             float av[2], dv2[2];
@@ -306,8 +313,10 @@ __device__ __forceinline__ void epi_block(const DevParams &p, const EpiBlock &e,
                     bias = e.tbs[bk];
                 }
                 int rraw = 0, ri;
-                if (DIRECT) {
+                if (KIND == 0) {
                     ri = e.rbase + cc;
+                } else if (KIND == 1) {
+                    ri = cc >= e.fc ? e.rc : e.rbase + cc;
                 } else {
                     rraw = min(i, e.Em1) - k.pj;
                     ri = rraw < 0 ? 0 : (rraw > p.R - 1 ? p.R - 1 : rraw);
@@ -326,7 +335,11 @@ __device__ __forceinline__ void epi_block(const DevParams &p, const EpiBlock &e,
                 dv2[q] = ds;
                 // ---- rel gradient: shift the diagonal sums one lane down, add this column
                 float vd = ds;
-                if (!DIRECT) {
+                if (KIND == 1) {
+                    const bool candc = cc >= e.fc;           // warp-uniform
+                    k.cand += candc ? ds : 0.f;
+                    vd = candc ? 0.f : ds;
+                } else if (KIND == 2) {
                     const bool candc = i > e.Em1;            // candidate row (warp-uniform)
                     const bool clamped = rraw != ri;
                     k.cand += candc ? ds : 0.f;
@@ -345,14 +358,23 @@ __device__ __forceinline__ void epi_block(const DevParams &p, const EpiBlock &e,
                     t_hi += bk ? ds : 0.f;
                     t_lo += bk ? 0.f : ds;
                 } else {
-                    const bool chg = valid && bk != k.cur_b;
-                    red_add_if(e.tb_slot + k.cur_b, k.run, chg && e.use_ts);
-                    k.cur_b = chg ? bk : k.cur_b;
-                    k.run = (chg ? 0.f : k.run) + ds;
+                    tbk[c] = valid ? bk : -1;
+                    tds[c] = ds;
                 }
             }
             pa[c2] = pack_bf16x2(av[0], av[1]);
             pd[c2] = pack_bf16x2(dv2[0], dv2[1]);
+        }
+        if (TM >= 2) {
+            // runs of equal buckets over the chunk's pairs, after all of its loads: a flush
+            // (inline asm) inside the pair loop would hold the next pairs' loads behind it
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const bool chg = tbk[c] >= 0 && tbk[c] != k.cur_b;
+                red_add_if(e.tb_slot + k.cur_b, k.run, chg && e.use_ts);
+                k.cur_b = chg ? tbk[c] : k.cur_b;
+                k.run = (chg ? 0.f : k.run) + tds[c];
+            }
         }
         tmem_st4(e.t_s + ch * 4, pa);
         st_shared_v4(e.ds_row + (((e.ds_chunk0 + ch) ^ e.rsw) << 4), pd[0], pd[1], pd[2], pd[3]);
@@ -740,18 +762,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                                          0u, 0u);
                         continue;
                     }
-                    // DIRECT blocks: every valid pair has rel index p(i) - p(j) = rbase + c
-                    // within the table and no candidate row (lanes without a valid pair
-                    // read the guarded table at base 0)
+                    // block kind (see epi_block): the history columns are direct when every
+                    // valid pair there has rel index p(i) - p(j) = rbase + c within the table
+                    // (lanes without a valid history pair read the guarded table at base 0)
                     const int fc = e.Em1 - e.iq + 1;           // first candidate column
                     const uint32_t candbits = fc >= QW ? 0u : (fc <= 0 ? ~0u : (~0u << fc));
                     const int rb = e.iq - k.pj;
-                    const int c_lo = __ffs(vb) - 1, c_hi = 31 - __clz(vb);
-                    const bool lane_direct =
-                        idle || ((vb & candbits) == 0u && rb + c_lo >= 0 && rb + c_hi <= p.R - 1);
-                    const bool direct =
-                        !use_rel || (rel_in_smem && __all_sync(0xffffffffu, lane_direct));
-                    e.rbase = (idle || !use_rel) ? 0 : rb;   // R = 0: all-zero guard band
+                    const uint32_t vh = vb & ~candbits;        // valid history columns
+                    const bool idle_h = vh == 0u;
+                    const int c_lo = __ffs(vh) - 1, c_hi = 31 - __clz(vh);
+                    const bool lane_ok = idle_h || (rb + c_lo >= 0 && rb + c_hi <= p.R - 1);
+                    const bool no_cand = __all_sync(0xffffffffu, (vb & candbits) == 0u);
+                    const bool all_ok =
+                        !use_rel || (rel_in_smem && __all_sync(0xffffffffu, lane_ok));
+                    // 0: direct, 1: direct with candidate columns, 2: general
+                    const int kind = !use_rel ? 0 : (all_ok ? (no_cand ? 0 : 1) : 2);
+                    e.rbase = (idle_h || !use_rel) ? 0 : rb;   // R = 0: all-zero guard band
+                    e.fc = fc;
+                    {
+                        const int rc = e.Em1 - k.pj;
+                        e.rc = rc < 0 ? 0 : (rc > p.R - 1 ? p.R - 1 : rc);
+                    }
                     e.tq32 = tsq32 + st * BM + wq * QW;
                     e.tq64 = tsq + st * BM + wq * QW;
                     HalfTime ht = {};
@@ -764,16 +795,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     float t_lo = 0.f, t_hi = 0.f;
                     tc_fence_after();
-                    if (direct) {
-                        if (tmode == 0) epi_block<0, true>(p, e, ht, k, t_lo, t_hi);
-                        else if (tmode == 1) epi_block<1, true>(p, e, ht, k, t_lo, t_hi);
-                        else if (tmode == 2) epi_block<2, true>(p, e, ht, k, t_lo, t_hi);
-                        else epi_block<3, false>(p, e, ht, k, t_lo, t_hi);
+                    if (tmode == 3) {
+                        epi_block<3, 2>(p, e, ht, k, t_lo, t_hi);
+                    } else if (kind == 0) {
+                        if (tmode == 0) epi_block<0, 0>(p, e, ht, k, t_lo, t_hi);
+                        else if (tmode == 1) epi_block<1, 0>(p, e, ht, k, t_lo, t_hi);
+                        else epi_block<2, 0>(p, e, ht, k, t_lo, t_hi);
+                    } else if (kind == 1) {
+                        if (tmode == 0) epi_block<0, 1>(p, e, ht, k, t_lo, t_hi);
+                        else if (tmode == 1) epi_block<1, 1>(p, e, ht, k, t_lo, t_hi);
+                        else epi_block<2, 1>(p, e, ht, k, t_lo, t_hi);
                     } else {
-                        if (tmode == 0) epi_block<0, false>(p, e, ht, k, t_lo, t_hi);
-                        else if (tmode == 1) epi_block<1, false>(p, e, ht, k, t_lo, t_hi);
-                        else if (tmode == 2) epi_block<2, false>(p, e, ht, k, t_lo, t_hi);
-                        else epi_block<3, false>(p, e, ht, k, t_lo, t_hi);
+                        if (tmode == 0) epi_block<0, 2>(p, e, ht, k, t_lo, t_hi);
+                        else if (tmode == 1) epi_block<1, 2>(p, e, ht, k, t_lo, t_hi);
+                        else epi_block<2, 2>(p, e, ht, k, t_lo, t_hi);
                     }
                     if (use_ts && tmode == 1) {
                         run_add(k, tb_slot, ht.blo, t_lo);
