@@ -289,11 +289,13 @@ hstu_status_t hstu_attn_bwd(const hstu_attn_params_t *p, const void *dout, const
     DevParams d = make_dev_params(p, seq_offsets, num_contextuals, num_targets, timestamps,
                                   rel_bias, time_bias, workspace);
     HSTU_CUDA_TRY(cudaMemsetAsync(workspace, 0, sizeof(int32_t), s));
-    if (p->rel_bias_len > 0)
-        HSTU_CUDA_TRY(cudaMemsetAsync(d_rel_bias, 0, sizeof(float) * p->rel_bias_len, s));
-    if (p->time_bias_len > 0)
-        HSTU_CUDA_TRY(cudaMemsetAsync(d_time_bias, 0, sizeof(float) * p->time_bias_len, s));
-    if (p->batch == 0 || p->total_tokens == 0) return HSTU_OK;
+    if (p->batch == 0 || p->total_tokens == 0) {
+        if (p->rel_bias_len > 0)
+            HSTU_CUDA_TRY(cudaMemsetAsync(d_rel_bias, 0, sizeof(float) * p->rel_bias_len, s));
+        if (p->time_bias_len > 0)
+            HSTU_CUDA_TRY(cudaMemsetAsync(d_time_bias, 0, sizeof(float) * p->time_bias_len, s));
+        return HSTU_OK;
+    }
 
     char *ws = reinterpret_cast<char *>(workspace) + kHeaderBytes;
     float *dy = reinterpret_cast<float *>(ws);
@@ -304,15 +306,22 @@ hstu_status_t hstu_attn_bwd(const hstu_attn_params_t *p, const void *dout, const
     float *dq_acc = f32 ? reinterpret_cast<float *>(dq) : reinterpret_cast<float *>(ws);
     float *tb_slots = f32 ? nullptr
                           : reinterpret_cast<float *>(ws + align_up((size_t)nq * 4, 256));
-    HSTU_CUDA_TRY(cudaMemsetAsync(dq_acc, 0, sizeof(float) * nq, s));
+    // the LayerNorm backward zeroes the dQ accumulator and the table gradients on its way
+    BwdZero zero;
+    zero.rows = dq_acc;
+    zero.row_floats = (int64_t)p->num_heads * p->d_qk;
+    zero.a = d_rel_bias;
+    zero.na = p->rel_bias_len;
+    zero.b = d_time_bias;
+    zero.nb = p->time_bias_len;
     {
         StageScope scope(HSTU_STAGE_BWD_NORM, s);
         if (f32)
             HSTU_CUDA_TRY(launch_ln_gate_bwd<float>(d, dout, u, saved_y, saved_mean, saved_rstd,
-                                                    du, dy, false, s));
+                                                    du, dy, false, zero, s));
         else
             HSTU_CUDA_TRY(launch_ln_gate_bwd<__nv_bfloat16>(d, dout, u, saved_y, saved_mean,
-                                                            saved_rstd, du, dy, tc, s));
+                                                            saved_rstd, du, dy, tc, zero, s));
     }
     {
         StageScope scope(HSTU_STAGE_BWD_ATTN, s);

@@ -15,12 +15,42 @@ cudaError_t launch_simt_fwd(const DevParams &p, const void *q, const void *k, co
 template <typename T>
 cudaError_t launch_ln_gate(const DevParams &p, const float *y, const void *u, void *out,
                            float *mean, float *rstd, cudaStream_t st);
+// Buffers the LayerNorm backward zeroes on the way, so that the attention backward that
+// follows on the stream needs no separate memset launches: row_floats floats per token at
+// rows (the dQ accumulator), and the two table-gradient arrays (by block 0).
+struct BwdZero {
+    float *rows;
+    int64_t row_floats;
+    float *a, *b;
+    int na, nb;
+};
+
+__device__ __forceinline__ void bwd_zero_row(const BwdZero &z, int64_t row, int lane)
+{
+    if (z.rows) {
+        float *r = z.rows + row * z.row_floats;
+        if ((z.row_floats & 3) == 0) {
+            float4 *r4 = reinterpret_cast<float4 *>(r);
+            for (int64_t x = lane; x < z.row_floats / 4; x += 32) r4[x] = make_float4(0.f, 0.f, 0.f, 0.f);
+        } else {
+            for (int64_t x = lane; x < z.row_floats; x += 32) r[x] = 0.f;
+        }
+    }
+}
+
+__device__ __forceinline__ void bwd_zero_small(const BwdZero &z)
+{
+    if (blockIdx.x != 0) return;
+    for (int x = threadIdx.x; x < z.na; x += blockDim.x) z.a[x] = 0.f;
+    for (int x = threadIdx.x; x < z.nb; x += blockDim.x) z.b[x] = 0.f;
+}
+
 // dy receives fp32 values (dy_bf16 false) or bf16 hi parts at dy and lo parts at dy + T*D
 // (dy_bf16 true).
 template <typename T>
 cudaError_t launch_ln_gate_bwd(const DevParams &p, const void *dout, const void *u,
                                const float *y, const float *mean, const float *rstd, void *du,
-                               void *dy, bool dy_bf16, cudaStream_t st);
+                               void *dy, bool dy_bf16, const BwdZero &zero, cudaStream_t st);
 // Vectorised LayerNorm + gating (norm.cu) for rows of 128*k features (k <= 8 or 16).
 bool ln_vec_supported(int D);
 template <typename T>
@@ -29,7 +59,8 @@ cudaError_t launch_ln_gate_vec(const DevParams &p, const float *y, const void *u
 template <typename T>
 cudaError_t launch_ln_gate_bwd_vec(const DevParams &p, const void *dout, const void *u,
                                    const float *y, const float *mean, const float *rstd,
-                                   void *du, void *dy, bool dy_bf16, cudaStream_t st);
+                                   void *du, void *dy, bool dy_bf16, const BwdZero &zero,
+                                   cudaStream_t st);
 template <typename T>
 cudaError_t launch_simt_bwd(const DevParams &p, const void *q, const void *k, const void *v,
                             const float *dy, float *dq_acc, void *dk, void *dv, float *d_rel,

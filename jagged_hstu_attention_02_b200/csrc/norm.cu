@@ -106,12 +106,14 @@ __global__ void __launch_bounds__(32 * kRows)
     ln_gate_bwd_vec_kernel(const __grid_constant__ DevParams p, const T *__restrict__ dout,
                            const T *__restrict__ u, const float *__restrict__ y,
                            const float *__restrict__ mean, const float *__restrict__ rstd,
-                           T *__restrict__ du, DYT *__restrict__ dy)
+                           T *__restrict__ du, DYT *__restrict__ dy, const BwdZero zj)
 {
     using V = Vec4<T>;
     const int lane = threadIdx.x & 31;
     const int64_t row = (int64_t)blockIdx.x * kRows + (threadIdx.x >> 5);
+    bwd_zero_small(zj);
     if (row >= p.T) return;
+    bwd_zero_row(zj, row, lane);
     constexpr int D = 128 * NV;
     const float mu = mean[row], rs = rstd[row];
     const float4 *yr = reinterpret_cast<const float4 *>(y + row * D) + lane;
@@ -175,15 +177,15 @@ cudaError_t fwd_nv(const DevParams &p, const float *y, const void *u, void *out,
 template <typename T, int NV>
 cudaError_t bwd_nv(const DevParams &p, const void *dout, const void *u, const float *y,
                    const float *mean, const float *rstd, void *du, void *dy, bool dy_bf16,
-                   cudaStream_t st)
+                   const BwdZero &zero, cudaStream_t st)
 {
     const int64_t blocks = (p.T + kRows - 1) / kRows;
     if (dy_bf16)
         ln_gate_bwd_vec_kernel<T, __nv_bfloat16, NV><<<(unsigned)blocks, 32 * kRows, 0, st>>>(
-            p, (const T *)dout, (const T *)u, y, mean, rstd, (T *)du, (__nv_bfloat16 *)dy);
+            p, (const T *)dout, (const T *)u, y, mean, rstd, (T *)du, (__nv_bfloat16 *)dy, zero);
     else
         ln_gate_bwd_vec_kernel<T, float, NV><<<(unsigned)blocks, 32 * kRows, 0, st>>>(
-            p, (const T *)dout, (const T *)u, y, mean, rstd, (T *)du, (float *)dy);
+            p, (const T *)dout, (const T *)u, y, mean, rstd, (T *)du, (float *)dy, zero);
     return cudaGetLastError();
 }
 
@@ -212,18 +214,19 @@ cudaError_t launch_ln_gate_vec(const DevParams &p, const float *y, const void *u
 template <typename T>
 cudaError_t launch_ln_gate_bwd_vec(const DevParams &p, const void *dout, const void *u,
                                    const float *y, const float *mean, const float *rstd,
-                                   void *du, void *dy, bool dy_bf16, cudaStream_t st)
+                                   void *du, void *dy, bool dy_bf16, const BwdZero &zero,
+                                   cudaStream_t st)
 {
     switch (p.D / 128) {
-    case 1: return bwd_nv<T, 1>(p, dout, u, y, mean, rstd, du, dy, dy_bf16, st);
-    case 2: return bwd_nv<T, 2>(p, dout, u, y, mean, rstd, du, dy, dy_bf16, st);
-    case 3: return bwd_nv<T, 3>(p, dout, u, y, mean, rstd, du, dy, dy_bf16, st);
-    case 4: return bwd_nv<T, 4>(p, dout, u, y, mean, rstd, du, dy, dy_bf16, st);
-    case 5: return bwd_nv<T, 5>(p, dout, u, y, mean, rstd, du, dy, dy_bf16, st);
-    case 6: return bwd_nv<T, 6>(p, dout, u, y, mean, rstd, du, dy, dy_bf16, st);
-    case 7: return bwd_nv<T, 7>(p, dout, u, y, mean, rstd, du, dy, dy_bf16, st);
-    case 8: return bwd_nv<T, 8>(p, dout, u, y, mean, rstd, du, dy, dy_bf16, st);
-    case 16: return bwd_nv<T, 16>(p, dout, u, y, mean, rstd, du, dy, dy_bf16, st);
+    case 1: return bwd_nv<T, 1>(p, dout, u, y, mean, rstd, du, dy, dy_bf16, zero, st);
+    case 2: return bwd_nv<T, 2>(p, dout, u, y, mean, rstd, du, dy, dy_bf16, zero, st);
+    case 3: return bwd_nv<T, 3>(p, dout, u, y, mean, rstd, du, dy, dy_bf16, zero, st);
+    case 4: return bwd_nv<T, 4>(p, dout, u, y, mean, rstd, du, dy, dy_bf16, zero, st);
+    case 5: return bwd_nv<T, 5>(p, dout, u, y, mean, rstd, du, dy, dy_bf16, zero, st);
+    case 6: return bwd_nv<T, 6>(p, dout, u, y, mean, rstd, du, dy, dy_bf16, zero, st);
+    case 7: return bwd_nv<T, 7>(p, dout, u, y, mean, rstd, du, dy, dy_bf16, zero, st);
+    case 8: return bwd_nv<T, 8>(p, dout, u, y, mean, rstd, du, dy, dy_bf16, zero, st);
+    case 16: return bwd_nv<T, 16>(p, dout, u, y, mean, rstd, du, dy, dy_bf16, zero, st);
     default: return cudaErrorInvalidValue;
     }
 }
@@ -236,10 +239,11 @@ template cudaError_t launch_ln_gate_vec<__nv_bfloat16>(const DevParams &, const 
 template cudaError_t launch_ln_gate_bwd_vec<float>(const DevParams &, const void *,
                                                    const void *, const float *, const float *,
                                                    const float *, void *, void *, bool,
-                                                   cudaStream_t);
+                                                   const BwdZero &, cudaStream_t);
 template cudaError_t launch_ln_gate_bwd_vec<__nv_bfloat16>(const DevParams &, const void *,
                                                            const void *, const float *,
                                                            const float *, const float *,
-                                                           void *, void *, bool, cudaStream_t);
+                                                           void *, void *, bool,
+                                                           const BwdZero &, cudaStream_t);
 
 }  // namespace hstu

@@ -245,11 +245,13 @@ __global__ void __launch_bounds__(kThreads)
     ln_gate_bwd_kernel(const __grid_constant__ DevParams p, const T *__restrict__ dout,
                        const T *__restrict__ u, const float *__restrict__ y,
                        const float *__restrict__ mean, const float *__restrict__ rstd,
-                       T *__restrict__ du, DYT *__restrict__ dy)
+                       T *__restrict__ du, DYT *__restrict__ dy, const BwdZero zj)
 {
     const int lane = threadIdx.x & 31;
     const int64_t row = (int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
+    bwd_zero_small(zj);
     if (row >= p.T) return;
+    bwd_zero_row(zj, row, lane);
     const int D = p.D;
     const float mu = mean[row], rs = rstd[row];
     float z[64], dz[64];
@@ -508,18 +510,18 @@ cudaError_t launch_ln_gate(const DevParams &p, const float *y, const void *u, vo
 template <typename T>
 cudaError_t launch_ln_gate_bwd(const DevParams &p, const void *dout, const void *u,
                                const float *y, const float *mean, const float *rstd, void *du,
-                               void *dy, bool dy_bf16, cudaStream_t st)
+                               void *dy, bool dy_bf16, const BwdZero &zero, cudaStream_t st)
 {
     if (ln_vec_supported(p.D))
-        return launch_ln_gate_bwd_vec<T>(p, dout, u, y, mean, rstd, du, dy, dy_bf16, st);
+        return launch_ln_gate_bwd_vec<T>(p, dout, u, y, mean, rstd, du, dy, dy_bf16, zero, st);
     const int rows_per_block = kThreads / 32;
     const int64_t blocks = (p.T + rows_per_block - 1) / rows_per_block;
     if (dy_bf16)
         ln_gate_bwd_kernel<T, __nv_bfloat16><<<(unsigned)blocks, kThreads, 0, st>>>(
-            p, (const T *)dout, (const T *)u, y, mean, rstd, (T *)du, (__nv_bfloat16 *)dy);
+            p, (const T *)dout, (const T *)u, y, mean, rstd, (T *)du, (__nv_bfloat16 *)dy, zero);
     else
         ln_gate_bwd_kernel<T, float><<<(unsigned)blocks, kThreads, 0, st>>>(
-            p, (const T *)dout, (const T *)u, y, mean, rstd, (T *)du, (float *)dy);
+            p, (const T *)dout, (const T *)u, y, mean, rstd, (T *)du, (float *)dy, zero);
     return cudaGetLastError();
 }
 
@@ -560,11 +562,13 @@ template cudaError_t launch_ln_gate<__nv_bfloat16>(const DevParams &, const floa
                                                    cudaStream_t);
 template cudaError_t launch_ln_gate_bwd<float>(const DevParams &, const void *, const void *,
                                                const float *, const float *, const float *,
-                                               void *, void *, bool, cudaStream_t);
+                                               void *, void *, bool, const BwdZero &,
+                                               cudaStream_t);
 template cudaError_t launch_ln_gate_bwd<__nv_bfloat16>(const DevParams &, const void *,
                                                        const void *, const float *,
                                                        const float *, const float *, void *,
-                                                       void *, bool, cudaStream_t);
+                                                       void *, bool, const BwdZero &,
+                                                       cudaStream_t);
 template cudaError_t launch_simt_bwd<float>(const DevParams &, const void *, const void *,
                                             const void *, const float *, float *, void *, void *,
                                             float *, float *, cudaStream_t);
