@@ -165,8 +165,12 @@ __device__ __forceinline__ HalfTime half_time_setup(const uint64_t *thr, int n_t
             dhi = a > c ? a : c;
         }
         if (lut_ok && dhi < (uint64_t)(INT32_MAX - 1)) {
+            // the bucket of dhi only matters as blo, blo + 1 or beyond: compare dhi with the
+            // next two thresholds instead of a second lookup (equal thresholds skip a bucket)
             h.blo = lut_bucket(lut, (uint32_t)dlo);
-            bhi = lut_bucket(lut, (uint32_t)dhi);
+            const uint64_t t1 = h.blo < n_thr ? thr[h.blo] : ~0ull;
+            const uint64_t t2 = h.blo + 1 < n_thr ? thr[h.blo + 1] : ~0ull;
+            bhi = dhi < t1 ? h.blo : (dhi < t2 ? h.blo + 1 : h.blo + 2);
         } else {
             h.blo = bucket_in(thr, 0, n_thr, dlo);
             bhi = bucket_in(thr, h.blo, n_thr, dhi);

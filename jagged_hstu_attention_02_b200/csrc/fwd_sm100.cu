@@ -559,8 +559,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 const int st = g & 1, ps = g % NP;
                 const int jq = t.kt * BN + wq * QW;      // first key of this warpgroup's quarter
                 const bool full = tile_all_valid(i0, i0 + BM - 1, jq, jq + QW - 1, s, p.W);
-                if (!warp_wait(&bars[META_FULL + st], (g >> 1) & 1) ||
-                    !warp_wait(&bars[S_FULL + st], (g >> 1) & 1)) {
+                // the set-up below needs only the stamps; S is waited for afterwards
+                if (!warp_wait(&bars[META_FULL + st], (g >> 1) & 1)) {
                     ok = false;
                     break;
                 }
@@ -596,8 +596,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 e.thr = thr;
                 e.n_thr = p.n_thr;
                 e.tsi = tsi;
-                // A's buffer is free once the A V of tile g - NP has completed
-                if (g >= NP && !warp_wait(&bars[P_FREE + ps], ((g / NP) - 1) & 1)) {
+                // S of this tile; A's buffer is free once the A V of tile g - NP has completed
+                if (!warp_wait(&bars[S_FULL + st], (g >> 1) & 1) ||
+                    (g >= NP && !warp_wait(&bars[P_FREE + ps], ((g / NP) - 1) & 1))) {
                     ok = false;
                     break;
                 }
