@@ -194,16 +194,16 @@ __device__ __forceinline__ void fwd_quarter(const FwdEpi &e, const HalfTime &ht,
     const uint32_t a1 = (uint32_t)ht.cmpA + 1u;
     const int64_t sp = (int64_t)ht.cmpB - (int64_t)ht.cmpA - 1;
     const uint32_t span = sp > 0 ? (uint32_t)sp : 0u;
-#pragma unroll
-    for (int hf = 0; hf < 2; ++hf) {
-        const int cb = hf * 16;
-        uint32_t ra[16];
-        tmem_ld16(e.t_s + cb, ra);
+#pragma unroll 1   // one copy of the 8-key body per mode combination (instruction cache)
+    for (int ch = 0; ch < 4; ++ch) {
+        const int cb = ch * 8;
+        uint32_t ra[8];
+        tmem_ld8(e.t_s + cb, ra);
         tmem_wait_ld();
         reg_fence(ra);
-        float bh[16];   // half of the bias
+        float bh[8];   // half of the bias
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
+        for (int c = 0; c < 8; ++c) {
             float tb;
             if (TM == 0) {
                 tb = ht.tb_lo;
@@ -225,12 +225,12 @@ __device__ __forceinline__ void fwd_quarter(const FwdEpi &e, const HalfTime &ht,
         }
         // SiLU(x) = x sigmoid(x) = h + h tanh(h), h = x/2; mask after the nonlinearity
         const uint32_t vb = vmask >> cb;
-        uint32_t pk[8];
+        uint32_t pk[4];
         if constexpr (SPLIT) {
             // training forward: accurate sigmoid in fp32, A split into hi + lo
-            uint32_t plo[8];
+            uint32_t plo[4];
 #pragma unroll
-            for (int c2 = 0; c2 < 8; ++c2) {
+            for (int c2 = 0; c2 < 4; ++c2) {
                 float a[2];
 #pragma unroll
                 for (int q = 0; q < 2; ++q) {
@@ -243,13 +243,13 @@ __device__ __forceinline__ void fwd_quarter(const FwdEpi &e, const HalfTime &ht,
                 plo[c2] = pack_bf16x2(a[0] - __uint_as_float(pk[c2] << 16),
                                       a[1] - __uint_as_float(pk[c2] & 0xFFFF0000u));
             }
-            tmem_st8(e.t_a + hf * 8, pk);
-            tmem_st8(e.t_a + 16 + hf * 8, plo);
+            tmem_st4(e.t_a + ch * 4, pk);
+            tmem_st4(e.t_a + 16 + ch * 4, plo);
         } else {
             // inference forward: h in fp32, then tanh and h + h tanh(h) on bf16 pairs
             // (A is rounded to bf16 for the tensor core either way)
 #pragma unroll
-            for (int c2 = 0; c2 < 8; ++c2) {
+            for (int c2 = 0; c2 < 4; ++c2) {
                 const float x0 = fmaf(e.half_alpha, __uint_as_float(ra[2 * c2]), bh[2 * c2]);
                 const float x1 = fmaf(e.half_alpha, __uint_as_float(ra[2 * c2 + 1]), bh[2 * c2 + 1]);
                 // bf16 pair = the high halves of x0, x1 (one byte permute)
@@ -260,7 +260,7 @@ __device__ __forceinline__ void fwd_quarter(const FwdEpi &e, const HalfTime &ht,
                           (((vb >> (2 * c2 + 1)) & 1u) ? 0xFFFF0000u : 0u);
                 pk[c2] = a2;
             }
-            tmem_st8(e.t_a + hf * 8, pk);
+            tmem_st4(e.t_a + ch * 4, pk);
         }
     }
 }
