@@ -466,8 +466,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     using L = BwdLayout<DQK, DV>;
     const DevParams &p = args.p;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                              ~static_cast<uintptr_t>(1023));
+    // 1024-byte aligned base, by an offset from the shared array (keeps the compiler aware
+    // that every table below lives in shared memory: 32-bit addresses, shared loads)
+    uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::BAR_OFF);
     uint32_t *slot = reinterpret_cast<uint32_t *>(sm + L::SLOT_OFF);
     int32_t *lut_valid = reinterpret_cast<int32_t *>(sm + L::SLOT_OFF + 4);
