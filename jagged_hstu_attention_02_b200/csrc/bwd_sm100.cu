@@ -23,8 +23,9 @@
 // memory retries under contention, and the pairs of one query hit few buckets):
 //   rel: within a 32-key x 32-query block the index is the diagonal i - j, so each warp sums
 //        the diagonals in registers by shifting partial sums one lane per column, and adds
-//        the 63 diagonal sums with two scatters; pairs whose index is clamped (candidate
-//        rows, far or bidirectional pairs) go to per-lane sums with one index each.
+//        the 63 diagonal sums with two scatters; candidate rows (index p(E-1) - p(j))
+//        go to a per-lane sum; the rare blocks with bidirectional contextual or
+//        out-of-table pairs add each pair into the output with a global reduction.
 //   time: along a key row the bucket changes rarely (timestamps ascend with position), so
 //        each lane sums runs of equal buckets and adds a run with one fire-and-forget global
 //        reduction into a histogram private to the CTA, folded into the output at the end.
@@ -216,9 +217,8 @@ struct KeyLane {
     bool key_in;
     int64_t tsj;
     // rel gradient: shifted diagonal sums (A: diagonals 31 - lane, B: -1 - lane of the
-    // 32 x 32 block) and the clamped pairs (candidate rows, index p(E-1) - p(j); negative
-    // distance, index 0; beyond the table, index R-1)
-    float sysA, sysB, cand, negs, fars;
+    // 32 x 32 block) and the candidate-row pairs (index p(E-1) - p(j))
+    float sysA, sysB, cand;
     // time gradient: the open run of equal buckets
     int cur_b;
     float run;
@@ -235,6 +235,7 @@ struct EpiBlock {
     int iq;                       // first query of the block
     int rbase;                    // p(iq) - p(j) in direct blocks (history columns)
     int fc, rc;                   // first candidate column; this key's rel index for it
+    float *d_rel;                 // the rel-gradient output (kind 2 adds into it directly)
     int Em1;                      // p(i) = min(i, Em1)
     bool full, use_rel, use_ts, rel_in_smem;
     uint32_t vbits;               // valid queries of this key (bit c <-> query iq + c)
@@ -253,7 +254,7 @@ struct EpiBlock {
 //      reads of masked pairs (at most 31 entries off) in bounds;
 //   1  direct for the history columns, and the candidate columns (c >= fc, p(i) = E - 1)
 //      at the lane's constant index rc;
-//   2  every index clamped, candidate / negative / out-of-table pairs sorted out per pair.
+//   2  every index clamped; each pair adds into the output directly (rare blocks).
 template <int TM, int KIND>
 __device__ __forceinline__ void epi_block(const DevParams &p, const EpiBlock &e,
                                           const HalfTime &ht, KeyLane &k, float &t_lo,
@@ -312,13 +313,13 @@ __device__ __forceinline__ void epi_block(const DevParams &p, const EpiBlock &e,
                     bk = bucket_search(e.thr, p.n_thr, abs_diff_u64(k.tsj, e.tq64[cc]));
                     bias = e.tbs[bk];
                 }
-                int rraw = 0, ri;
+                int ri;
                 if (KIND == 0) {
                     ri = e.rbase + cc;
                 } else if (KIND == 1) {
                     ri = cc >= e.fc ? e.rc : e.rbase + cc;
                 } else {
-                    rraw = min(i, e.Em1) - k.pj;
+                    const int rraw = min(i, e.Em1) - k.pj;
                     ri = rraw < 0 ? 0 : (rraw > p.R - 1 ? p.R - 1 : rraw);
                 }
                 bias += e.relp[ri];
@@ -340,17 +341,16 @@ __device__ __forceinline__ void epi_block(const DevParams &p, const EpiBlock &e,
                     k.cand += candc ? ds : 0.f;
                     vd = candc ? 0.f : ds;
                 } else if (KIND == 2) {
-                    const bool candc = i > e.Em1;            // candidate row (warp-uniform)
-                    const bool clamped = rraw != ri;
-                    k.cand += candc ? ds : 0.f;
-                    k.negs += (!candc && clamped && rraw < 0) ? ds : 0.f;
-                    k.fars += (!candc && clamped && rraw >= 0) ? ds : 0.f;
-                    vd = (candc || clamped) ? 0.f : ds;
+                    // rare blocks (bidirectional contextual or out-of-table pairs): every
+                    // pair, masked ones adding zero, straight into the output at its index
+                    atomicAdd(e.d_rel + ri, ds);
                 }
-                const float ain = __shfl_sync(0xffffffffu, k.sysA, src);
-                const float bin = __shfl_sync(0xffffffffu, k.sysB, src);
-                k.sysB = lane0 ? ain : bin;
-                k.sysA = (lane0 ? 0.f : ain) + vd;
+                if (KIND != 2) {
+                    const float ain = __shfl_sync(0xffffffffu, k.sysA, src);
+                    const float bin = __shfl_sync(0xffffffffu, k.sysB, src);
+                    k.sysB = lane0 ? ain : bin;
+                    k.sysA = (lane0 ? 0.f : ain) + vd;
+                }
                 // ---- time gradient
                 if (TM == 0) {
                     k.run += ds;
@@ -396,18 +396,7 @@ __device__ __forceinline__ void flush_rel(const DevParams &p, KeyLane &k, int iq
         rc = rc < 0 ? 0 : (rc > p.R - 1 ? p.R - 1 : rc);
         rel_add(hrel, d_rel, in_smem, rc, k.cand);
     }
-    if (__any_sync(0xffffffffu, k.negs != 0.f || k.fars != 0.f)) {
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            k.negs += __shfl_xor_sync(0xffffffffu, k.negs, o);
-            k.fars += __shfl_xor_sync(0xffffffffu, k.fars, o);
-        }
-        if (lane == 0) {
-            if (k.negs != 0.f) rel_add(hrel, d_rel, in_smem, 0, k.negs);
-            if (k.fars != 0.f) rel_add(hrel, d_rel, in_smem, p.R - 1, k.fars);
-        }
-    }
-    k.sysA = k.sysB = k.cand = k.negs = k.fars = 0.f;
+    k.sysA = k.sysB = k.cand = 0.f;
 }
 
 // Adds v to the time-gradient run state for bucket b (closing the open run if it differs).
@@ -716,6 +705,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         e.tbs = tbs;
         e.lut = lut;
         e.tb_slot = tb_slot;
+        e.d_rel = args.d_rel;
         UnitIter un(p, args.nkt, false);
         int n = 0, g = 0;
         bool ok = true;
@@ -727,7 +717,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             k.key_in = k.j < s.L;
             k.pj = clamp_pos(k.j, s.E);
             k.tsj = (use_ts && k.key_in) ? p.ts[s.start + k.pj] : 0;
-            k.sysA = k.sysB = k.cand = k.negs = k.fars = 0.f;
+            k.sysA = k.sysB = k.cand = 0.f;
             k.cur_b = 0;
             k.run = 0.f;
             e.Em1 = s.E > 0 ? s.E - 1 : 0x7fffffff;
