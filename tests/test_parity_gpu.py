@@ -256,3 +256,45 @@ def test_bad_device_data_is_reported_and_the_context_stays_usable():
     assert ops.read_device_status(ops.fwd.last_workspace) & ops.DEV_SEQ_TOO_LONG
     # a valid call afterwards still matches the oracle
     _fwd_check(b, what="after bad data")
+
+
+# ------------------------------------------------------------------ timestamp orders and ranges
+#
+# The workloads draw ascending timestamps; the kernels exploit ascending order only for
+# speed (runs of equal buckets, one-boundary blocks).  Any order and any range is an input
+# the library must get right: shuffled stamps inside each sequence, and gaps beyond 2^31
+# that force the 64-bit bucket search.
+
+def _stamped(seed, stamps, dqk=128, dv=128):
+    lengths = [130, 300, 77, 256]
+    b = synth.make_batch(np.random.default_rng(seed), lengths, 2, dqk, dv, "bf16",
+                         contextuals=[1, 4, 0, 3], targets=[5, 40, 2, 0], rel_bias_len=301,
+                         time_bias_len=128, with_dout=True)
+    rng = np.random.default_rng(seed + 1)
+    ts = b.timestamps.copy()
+    for s in range(b.batch):
+        a, e = int(b.seq_offsets[s]), int(b.seq_offsets[s + 1])
+        if stamps == "shuffled":
+            ts[a:e] = rng.permutation(ts[a:e])
+        elif stamps == "huge-gaps":
+            gaps = rng.choice([1, 3600, 1 << 33, 7 << 40], size=e - a, p=[0.3, 0.4, 0.2, 0.1])
+            ts[a:e] = 1_000_000_000 + np.cumsum(gaps)
+    import dataclasses
+    return dataclasses.replace(b, timestamps=ts)
+
+
+@pytest.mark.parametrize("stamps", ["shuffled", "huge-gaps"])
+@pytest.mark.parametrize("dims", [(128, 128), (64, 64)])
+def test_fwd_bwd_parity_any_timestamp_order(stamps, dims):
+    b = _stamped(300, stamps, *dims)
+    name = "%s d=%s" % (stamps, dims)
+    _fwd_check(b, training=False, what=name + " inference")
+    dev = ops.batch_to_device(b)
+    out, saved = ops.run_fwd(b, dev, training=True)
+    dq, dk, dv_, du, drel, dtb = ops.run_bwd(b, saved, dev_tensors=dev)
+    torch.cuda.synchronize()
+    assert ops.read_device_status(ops.bwd.last_workspace) == 0
+    ref = oracle.bwd(b)
+    for got, key in ((dq, "dq"), (dk, "dk"), (dv_, "dv"), (du, "du"), (drel, "drel"),
+                     (dtb, "dtb")):
+        assert_close(_np(got), ref[key], "bf16", name + " " + key)
