@@ -26,11 +26,9 @@ constexpr int kLutCells = 1024;
 
 __device__ __forceinline__ int lut_cell(uint32_t dt)
 {
-    const uint32_t y = dt + 1u;
-    const bool big = y >= (1u << 23);
-    const uint32_t ys = big ? (y >> 8) : y;                 // < 2^23: exact in fp32
-    const float f = __uint_as_float(0x4B000000u | ys) - 8388608.0f;
-    return (int)(__float_as_uint(f) >> 18) - (127 << 5) + (big ? (8 << 5) : 0);
+    // converted toward zero, y keeps its exponent and its leading mantissa bits exactly
+    const float f = __uint2float_rz(dt + 1u);
+    return (int)(__float_as_uint(f) >> 18) - (127 << 5);
 }
 
 // Bucket of dt known to lie in [lo, hi]: number of thresholds <= dt (thr[k-1] opens bucket k).
