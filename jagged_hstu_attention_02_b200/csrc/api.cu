@@ -15,7 +15,7 @@ namespace hstu {
 
 namespace {
 
-constexpr size_t kHeaderBytes = 256;   // status word + padding at the start of the workspace
+constexpr size_t kHeaderBytes = 256;   // status word, work-unit counter, padding
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -288,7 +288,8 @@ hstu_status_t hstu_attn_bwd(const hstu_attn_params_t *p, const void *dout, const
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     DevParams d = make_dev_params(p, seq_offsets, num_contextuals, num_targets, timestamps,
                                   rel_bias, time_bias, workspace);
-    HSTU_CUDA_TRY(cudaMemsetAsync(workspace, 0, sizeof(int32_t), s));
+    // status word (bytes 0-3) and the work-unit counter (bytes 8-15) of the header
+    HSTU_CUDA_TRY(cudaMemsetAsync(workspace, 0, 16, s));
     if (p->batch == 0 || p->total_tokens == 0) {
         if (p->rel_bias_len > 0)
             HSTU_CUDA_TRY(cudaMemsetAsync(d_rel_bias, 0, sizeof(float) * p->rel_bias_len, s));
@@ -329,8 +330,10 @@ hstu_status_t hstu_attn_bwd(const hstu_attn_params_t *p, const void *dout, const
             HSTU_CUDA_TRY(launch_simt_bwd<float>(d, q, k, v, dy, dq_acc, dk, dv, d_rel_bias,
                                                  d_time_bias, s));
         } else if (tc) {
-            HSTU_CUDA_TRY(launch_tc_bwd(d, q, k, v, dy, dq_acc, dk, dv, d_rel_bias, d_time_bias,
-                                        tb_slots, s));
+            HSTU_CUDA_TRY(launch_tc_bwd(
+                d, q, k, v, dy, dq_acc, dk, dv, d_rel_bias, d_time_bias, tb_slots,
+                reinterpret_cast<unsigned long long *>(reinterpret_cast<char *>(workspace) + 8),
+                s));
             HSTU_CUDA_TRY(launch_convert<__nv_bfloat16>(dq_acc, dq, nq, s));
         } else {
             HSTU_CUDA_TRY(launch_simt_bwd<__nv_bfloat16>(d, q, k, v, dy, dq_acc, dk, dv,

@@ -61,8 +61,10 @@ enum Bar {
     KV_FULL = 0, KV_EMPTY = 1, QD_FULL = 2, QD_EMPTY = 3, SD_FULL = 4, META_FULL = 5,  // +2
     EPI_DONE = 7,                                                                     // +2
     P_FULL = 9, DQ_FULL = 10, DQ_FREE = 11, ACC_FULL = 12, ACC_FREE = 13, MMA_DONE = 14,
-    NUM_BARS = 15
+    UNIT_FULL = 15, UNIT_EMPTY = 19,                                                  // +4
+    NUM_BARS = 23
 };
+constexpr int kRing = 4;                // work units published ahead by the producer
 
 // Time-stamp ranges of the four 32-query quarters of a query tile.
 struct QMeta {
@@ -84,8 +86,9 @@ struct BwdLayout {
     static constexpr int Y_OFF = Q_OFF + QB;
     static constexpr int YL_OFF = Y_OFF + YB;     // also DS
     static constexpr int BAR_OFF = YL_OFF + LB;
-    static constexpr int SLOT_OFF = BAR_OFF + 8 * 16;
-    static constexpr int META_OFF = SLOT_OFF + 16;
+    static constexpr int SLOT_OFF = BAR_OFF + 8 * 32;
+    static constexpr int UNIT_OFF = SLOT_OFF + 16;                 // kRing unit indices
+    static constexpr int META_OFF = UNIT_OFF + 8 * kRing;
     static constexpr int TSQ_OFF = META_OFF + 2 * (int)sizeof(QMeta);
     static constexpr int TSQ32_OFF = TSQ_OFF + 2 * BM * 8;
     static constexpr int LUT_OFF = TSQ32_OFF + 2 * BM * 4;
@@ -95,7 +98,7 @@ struct BwdLayout {
     static constexpr int HREL_OFF = REL_OFF + 4 * (kRelSmemMax + 2 * kRelGuard);
     static constexpr int TOTAL = HREL_OFF + 4 * kRelSmemMax;
     static constexpr int ALLOC = TOTAL + 1024;
-    static_assert(NUM_BARS <= 16, "barrier area");
+    static_assert(NUM_BARS <= 32, "barrier area");
     static_assert(TSQ_OFF % 8 == 0 && LUT_OFF % 8 == 0, "alignment");
 };
 
@@ -106,34 +109,86 @@ struct BwdTcArgs {
     __nv_bfloat16 *dk, *dv;        // [T, H, d]
     float *d_rel, *d_tb;
     float *tb_slots;               // [gridDim.x, kMaxTimeBuckets] scratch, one row per CTA
+    unsigned long long *unit_ctr;  // next work unit to hand out (zeroed by the caller)
     int nkt;                       // key tiles of the longest admissible sequence
 };
 
-// Work units (key tile kt, sequence b, head h), key tile 0 first: a unit over key tile kt
-// visits the query tiles kt .. of its sequence, so low kt carries the most work.
-struct UnitIter {
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity)
+{
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity));
+}
+
+// One arrival per warp on `bar` (counted per warp), after the whole warp got here.
+__device__ __forceinline__ void warp_arrive(uint64_t *bar)
+{
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+}
+
+// Work units (key tile kt, sequence b, head h), numbered key tile 0 first: a unit over key
+// tile kt visits the query tiles kt .. of its sequence, so low numbers carry the most work.
+// Units are handed out dynamically: the producer takes the next number from a global
+// counter (skipping units past a sequence's end) and publishes it in a ring of kRing slots
+// in shared memory; the MMA issuer, the stamp warp and the epilogue warps read the ring in
+// order.  A CTA that drew cheap units simply draws more, so the CTAs finish together.
+struct UnitFeed {
     const DevParams &p;
-    int nkt;
-    int64_t u, total;
-    bool report;
+    uint64_t *full, *empty;      // kRing barriers each
+    int64_t *slots;
+    unsigned long long *ctr;
+    int64_t total;
+    int role;                    // 0 producer thread, 1 consumer thread, 2 consumer warp
+    int k = 0;                   // units taken so far
+    bool ok = true;              // false once a bounded wait gave up
     SeqInfo s;
-    int kt, b, h;
-    __device__ UnitIter(const DevParams &p_, int nkt_, bool report_)
-        : p(p_), nkt(nkt_), u((int64_t)blockIdx.x - gridDim.x),
-          total((int64_t)nkt_ * p_.B * p_.H), report(report_) {}
+    int kt = 0, b = 0, h = 0;
+    __device__ UnitFeed(const DevParams &p_, uint64_t *bars, int64_t *slots_,
+                        unsigned long long *ctr_, int nkt, int role_)
+        : p(p_), full(bars + UNIT_FULL), empty(bars + UNIT_EMPTY), slots(slots_), ctr(ctr_),
+          total((int64_t)nkt * p_.B * p_.H), role(role_) {}
+    __device__ void decode(int64_t u)
+    {
+        const int64_t bh = (int64_t)p.B * p.H;
+        kt = (int)(u / bh);
+        const int rem = (int)(u % bh);
+        b = rem / p.H;
+        h = rem % p.H;
+    }
     __device__ bool next()
     {
-        while ((u += gridDim.x) < total) {
-            const int64_t bh = (int64_t)p.B * p.H;
-            kt = (int)(u / bh);
-            const int rem = (int)(u % bh);
-            b = rem / p.H;
-            h = rem % p.H;
-            if (!seq_may_have_tile(p, b, kt)) continue;
-            s = load_seq(p, b, report && kt == 0 && h == 0);
-            if (kt * BN < s.L) return true;
+        const int sl = k % kRing;
+        int64_t u = -1;
+        if (role == 0) {
+            while (true) {
+                const int64_t x = (int64_t)atomicAdd(ctr, 1ull);
+                if (x >= total) break;
+                decode(x);
+                if (!seq_may_have_tile(p, b, kt)) continue;
+                s = load_seq(p, b, false);
+                if (kt * BN < s.L) { u = x; break; }
+            }
+            if (k >= kRing && !mbar_wait(&empty[sl], ((k / kRing) - 1) & 1)) {
+                ok = false;
+                return false;
+            }
+            slots[sl] = u;
+            mbar_arrive(&full[sl]);      // releases the slot's contents
+            ++k;
+            return u >= 0;
         }
-        return false;
+        const bool got = role == 2 ? warp_wait(&full[sl], (k / kRing) & 1)
+                                   : mbar_wait(&full[sl], (k / kRing) & 1);
+        if (!got) {
+            ok = false;
+            return false;
+        }
+        u = *reinterpret_cast<volatile int64_t *>(&slots[sl]);
+        if (role == 2) warp_arrive(&empty[sl]); else mbar_arrive(&empty[sl]);
+        ++k;
+        if (u < 0) return false;
+        decode(u);
+        s = load_seq(p, b, false);
+        return true;
     }
 };
 
@@ -156,17 +211,6 @@ __device__ __forceinline__ void report_timeout(const DevParams &p)
     flag_error(p, HSTU_DEV_WAIT_TIMEOUT);
 }
 
-__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity)
-{
-    return __all_sync(0xffffffffu, mbar_wait(bar, parity));
-}
-
-// One arrival per warp on `bar` (counted per warp), after the whole warp got here.
-__device__ __forceinline__ void warp_arrive(uint64_t *bar)
-{
-    __syncwarp();
-    if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
-}
 
 __device__ __forceinline__ void red_add_v4(float *addr, float a, float b, float c, float d)
 {
@@ -461,6 +505,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::BAR_OFF);
     uint32_t *slot = reinterpret_cast<uint32_t *>(sm + L::SLOT_OFF);
     int32_t *lut_valid = reinterpret_cast<int32_t *>(sm + L::SLOT_OFF + 4);
+    int64_t *unit_slots = reinterpret_cast<int64_t *>(sm + L::UNIT_OFF);
     QMeta *meta = reinterpret_cast<QMeta *>(sm + L::META_OFF);
     int64_t *tsq = reinterpret_cast<int64_t *>(sm + L::TSQ_OFF);
     int32_t *tsq32 = reinterpret_cast<int32_t *>(sm + L::TSQ32_OFF);
@@ -479,6 +524,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&bars[P_FULL], kEpiWarps);
         mbar_init(&bars[DQ_FREE], kEpiWarps);
         mbar_init(&bars[ACC_FREE], kEpiWarps);
+        for (int x = 0; x < kRing; ++x) mbar_init(&bars[UNIT_EMPTY + x], 2 + kEpiWarps);
         fence_mbar_init();
         *lut_valid = 1;
     }
@@ -517,7 +563,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             prefetch_tmap(&args.tv);
             prefetch_tmap(&args.tdy);
             prefetch_tmap(&args.tdyl);
-            UnitIter un(p, args.nkt, true);
+            UnitFeed un(p, bars, unit_slots, args.unit_ctr, args.nkt, 0);
             int n = 0, g = 0;
             bool ok = true;
             while (ok && un.next()) {
@@ -548,7 +594,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ++g;
                 }
             }
-            if (!ok) report_timeout(p);
+            if (!ok || !un.ok) report_timeout(p);
             // every copy has landed before the CTA may exit
             bool drained = true;
             if (n >= 1) drained &= mbar_wait(&bars[KV_FULL], (n - 1) & 1);
@@ -565,7 +611,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t k_addr = sm_base + L::K_OFF, v_addr = sm_base + L::V_OFF;
             const uint32_t q_addr = sm_base + L::Q_OFF, y_addr = sm_base + L::Y_OFF;
             const uint32_t yl_addr = sm_base + L::YL_OFF, ds_addr = sm_base + L::YL_OFF;
-            UnitIter un(p, args.nkt, false);
+            UnitFeed un(p, bars, unit_slots, args.unit_ctr, args.nkt, 1);
             int n = 0, g = 0;
             bool ok = true;
             while (ok && un.next()) {
@@ -637,14 +683,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 umma_commit(&bars[ACC_FULL]);
                 ++n;
             }
-            if (!ok) report_timeout(p);
+            if (!ok || !un.ok) report_timeout(p);
             umma_commit(&bars[MMA_DONE]);
             if (!mbar_wait(&bars[MMA_DONE], 0)) report_timeout(p);
         }
     } else if (warp == 2) {
         // -------------------------------------------------------------------- query stamps
         const bool use_ts = p.NB > 0;
-        UnitIter un(p, args.nkt, false);
+        UnitFeed un(p, bars, unit_slots, args.unit_ctr, args.nkt, 2);
         int g = 0;
         bool ok = true;
         while (ok && un.next()) {
@@ -685,7 +731,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ++g;
             }
         }
-        if (!ok) report_timeout(p);
+        if (!ok || !un.ok) report_timeout(p);
     } else if (warp >= kEpiWarp0) {
         // -------------------------------------------------------------------- epilogue
         constexpr int kGroups = kEpiWarps / 4;        // warpgroups
@@ -706,7 +752,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         e.lut = lut;
         e.tb_slot = tb_slot;
         e.d_rel = args.d_rel;
-        UnitIter un(p, args.nkt, false);
+        UnitFeed un(p, bars, unit_slots, args.unit_ctr, args.nkt, 2);
         int n = 0, g = 0;
         bool ok = true;
         while (ok && un.next()) {
@@ -872,7 +918,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             ++n;
         }
-        if (!ok) report_timeout(p);
+        if (!ok || !un.ok) report_timeout(p);
     }
 
     tc_fence_before();
@@ -917,7 +963,8 @@ bool tc_bwd_supported(int dqk, int dv, int64_t T) { return tc_fwd_supported(dqk,
 
 cudaError_t launch_tc_bwd(const DevParams &p, const void *q, const void *k, const void *v,
                           const void *dy_bf16, float *dq_acc, void *dk, void *dv, float *d_rel,
-                          float *d_tb, float *tb_slots, cudaStream_t st)
+                          float *d_tb, float *tb_slots, unsigned long long *unit_ctr,
+                          cudaStream_t st)
 {
     BwdTcArgs a;
     std::memset(&a, 0, sizeof(a));
@@ -928,6 +975,7 @@ cudaError_t launch_tc_bwd(const DevParams &p, const void *q, const void *k, cons
     a.d_rel = d_rel;
     a.d_tb = d_tb;
     a.tb_slots = tb_slots;
+    a.unit_ctr = unit_ctr;
     a.nkt = (p.N + BN - 1) / BN;
     const void *dy_lo = reinterpret_cast<const char *>(dy_bf16) + (size_t)p.T * p.D * 2;
     if (!encode_tmap_bf16(&a.tq, q, p.dqk, p.H, p.T) || !encode_tmap_bf16(&a.tk, k, p.dqk, p.H, p.T) ||

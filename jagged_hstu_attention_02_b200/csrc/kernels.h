@@ -85,7 +85,7 @@ bool tc_bwd_supported(int dqk, int dv, int64_t T);
 cudaError_t launch_tc_bwd(const DevParams &p, const void *q, const void *k, const void *v,
                           const void *dy_bf16 /* hi, then lo at + T*D */, float *dq_acc,
                           void *dk, void *dv, float *d_rel, float *d_tb, float *tb_slots,
-                          cudaStream_t st);
+                          unsigned long long *unit_ctr /* zeroed */, cudaStream_t st);
 
 // [T, H, d] bf16 row-major as a 3-D TMA tensor (d, H, T): box 64 x 1 x 128, 128-byte swizzle.
 bool encode_tmap_bf16(CUtensorMap *m, const void *base, int d, int H, int64_t T);
