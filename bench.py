@@ -36,8 +36,8 @@ SECONDARY_CFG = 2         # long-history forward (tensor-core regime)
 # only while the kernel's sources hash to the value recorded with the capture.
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 KERNEL_SOURCES = {
-    "bwd_attn": ["bwd_sm100.cu", "bias.cuh", "common.cuh", "sm100.cuh"],
-    "fwd_attn": ["fwd_sm100.cu", "bias.cuh", "common.cuh", "sm100.cuh"],
+    "bwd_attn": ["bwd_sm100.cu", "bias.cuh", "common.cuh", "sm100.cuh", "units.cuh"],
+    "fwd_attn": ["fwd_sm100.cu", "bias.cuh", "common.cuh", "sm100.cuh", "units.cuh"],
 }
 
 

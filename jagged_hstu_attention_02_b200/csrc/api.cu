@@ -238,7 +238,8 @@ hstu_status_t hstu_attn_fwd(const hstu_attn_params_t *p, const void *q, const vo
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     DevParams d = make_dev_params(p, seq_offsets, num_contextuals, num_targets, timestamps,
                                   rel_bias, time_bias, workspace);
-    HSTU_CUDA_TRY(cudaMemsetAsync(workspace, 0, sizeof(int32_t), s));
+    // status word (bytes 0-3) and the work-unit counter (bytes 8-15) of the header
+    HSTU_CUDA_TRY(cudaMemsetAsync(workspace, 0, 16, s));
     if (p->batch == 0 || p->total_tokens == 0) return HSTU_OK;
     float *y = train ? saved_y
                      : reinterpret_cast<float *>(reinterpret_cast<char *>(workspace) + kHeaderBytes);
@@ -247,7 +248,10 @@ hstu_status_t hstu_attn_fwd(const hstu_attn_params_t *p, const void *q, const vo
         if (p->dtype == HSTU_F32)
             HSTU_CUDA_TRY(launch_simt_fwd<float>(d, q, k, v, y, s));
         else if (tc_fwd_supported(p->d_qk, p->d_v, p->total_tokens))
-            HSTU_CUDA_TRY(launch_tc_fwd(d, q, k, v, y, train, s));
+            HSTU_CUDA_TRY(launch_tc_fwd(
+                d, q, k, v, y,
+                reinterpret_cast<unsigned long long *>(reinterpret_cast<char *>(workspace) + 8),
+                train, s));
         else
             HSTU_CUDA_TRY(launch_simt_fwd<__nv_bfloat16>(d, q, k, v, y, s));
     }

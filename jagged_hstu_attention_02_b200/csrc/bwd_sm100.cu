@@ -38,6 +38,7 @@
 #include "bias.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
+#include "units.cuh"
 
 namespace hstu {
 
@@ -64,7 +65,6 @@ enum Bar {
     UNIT_FULL = 15, UNIT_EMPTY = 19,                                                  // +4
     NUM_BARS = 23
 };
-constexpr int kRing = 4;                // work units published ahead by the producer
 
 // Time-stamp ranges of the four 32-query quarters of a query tile.
 struct QMeta {
@@ -87,8 +87,8 @@ struct BwdLayout {
     static constexpr int YL_OFF = Y_OFF + YB;     // also DS
     static constexpr int BAR_OFF = YL_OFF + LB;
     static constexpr int SLOT_OFF = BAR_OFF + 8 * 32;
-    static constexpr int UNIT_OFF = SLOT_OFF + 16;                 // kRing unit indices
-    static constexpr int META_OFF = UNIT_OFF + 8 * kRing;
+    static constexpr int UNIT_OFF = SLOT_OFF + 16;                 // kUnitRing unit indices
+    static constexpr int META_OFF = UNIT_OFF + 8 * kUnitRing;
     static constexpr int TSQ_OFF = META_OFF + 2 * (int)sizeof(QMeta);
     static constexpr int TSQ32_OFF = TSQ_OFF + 2 * BM * 8;
     static constexpr int LUT_OFF = TSQ32_OFF + 2 * BM * 4;
@@ -111,85 +111,6 @@ struct BwdTcArgs {
     float *tb_slots;               // [gridDim.x, kMaxTimeBuckets] scratch, one row per CTA
     unsigned long long *unit_ctr;  // next work unit to hand out (zeroed by the caller)
     int nkt;                       // key tiles of the longest admissible sequence
-};
-
-__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity)
-{
-    return __all_sync(0xffffffffu, mbar_wait(bar, parity));
-}
-
-// One arrival per warp on `bar` (counted per warp), after the whole warp got here.
-__device__ __forceinline__ void warp_arrive(uint64_t *bar)
-{
-    __syncwarp();
-    if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
-}
-
-// Work units (key tile kt, sequence b, head h), numbered key tile 0 first: a unit over key
-// tile kt visits the query tiles kt .. of its sequence, so low numbers carry the most work.
-// Units are handed out dynamically: the producer takes the next number from a global
-// counter (skipping units past a sequence's end) and publishes it in a ring of kRing slots
-// in shared memory; the MMA issuer, the stamp warp and the epilogue warps read the ring in
-// order.  A CTA that drew cheap units simply draws more, so the CTAs finish together.
-struct UnitFeed {
-    const DevParams &p;
-    uint64_t *full, *empty;      // kRing barriers each
-    int64_t *slots;
-    unsigned long long *ctr;
-    int64_t total;
-    int role;                    // 0 producer thread, 1 consumer thread, 2 consumer warp
-    int k = 0;                   // units taken so far
-    bool ok = true;              // false once a bounded wait gave up
-    SeqInfo s;
-    int kt = 0, b = 0, h = 0;
-    __device__ UnitFeed(const DevParams &p_, uint64_t *bars, int64_t *slots_,
-                        unsigned long long *ctr_, int nkt, int role_)
-        : p(p_), full(bars + UNIT_FULL), empty(bars + UNIT_EMPTY), slots(slots_), ctr(ctr_),
-          total((int64_t)nkt * p_.B * p_.H), role(role_) {}
-    __device__ void decode(int64_t u)
-    {
-        const int64_t bh = (int64_t)p.B * p.H;
-        kt = (int)(u / bh);
-        const int rem = (int)(u % bh);
-        b = rem / p.H;
-        h = rem % p.H;
-    }
-    __device__ bool next()
-    {
-        const int sl = k % kRing;
-        int64_t u = -1;
-        if (role == 0) {
-            while (true) {
-                const int64_t x = (int64_t)atomicAdd(ctr, 1ull);
-                if (x >= total) break;
-                decode(x);
-                if (!seq_may_have_tile(p, b, kt)) continue;
-                s = load_seq(p, b, false);
-                if (kt * BN < s.L) { u = x; break; }
-            }
-            if (k >= kRing && !mbar_wait(&empty[sl], ((k / kRing) - 1) & 1)) {
-                ok = false;
-                return false;
-            }
-            slots[sl] = u;
-            mbar_arrive(&full[sl]);      // releases the slot's contents
-            ++k;
-            return u >= 0;
-        }
-        const bool got = role == 2 ? warp_wait(&full[sl], (k / kRing) & 1)
-                                   : mbar_wait(&full[sl], (k / kRing) & 1);
-        if (!got) {
-            ok = false;
-            return false;
-        }
-        u = *reinterpret_cast<volatile int64_t *>(&slots[sl]);
-        if (role == 2) warp_arrive(&empty[sl]); else mbar_arrive(&empty[sl]);
-        ++k;
-        if (u < 0) return false;
-        decode(u);
-        s = load_seq(p, b, false);
-        return true;
-    }
 };
 
 // The query tiles [i0, i0+BM) that see key tile [j0, j0+BN), in order.
@@ -505,7 +426,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::BAR_OFF);
     uint32_t *slot = reinterpret_cast<uint32_t *>(sm + L::SLOT_OFF);
     int32_t *lut_valid = reinterpret_cast<int32_t *>(sm + L::SLOT_OFF + 4);
-    int64_t *unit_slots = reinterpret_cast<int64_t *>(sm + L::UNIT_OFF);
+    // Work units: key tiles from the first up (the most query tiles first), sequence, head.
+    const FeedRing ring{bars + UNIT_FULL, bars + UNIT_EMPTY,
+                        reinterpret_cast<int64_t *>(sm + L::UNIT_OFF), args.unit_ctr};
     QMeta *meta = reinterpret_cast<QMeta *>(sm + L::META_OFF);
     int64_t *tsq = reinterpret_cast<int64_t *>(sm + L::TSQ_OFF);
     int32_t *tsq32 = reinterpret_cast<int32_t *>(sm + L::TSQ32_OFF);
@@ -524,7 +447,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&bars[P_FULL], kEpiWarps);
         mbar_init(&bars[DQ_FREE], kEpiWarps);
         mbar_init(&bars[ACC_FREE], kEpiWarps);
-        for (int x = 0; x < kRing; ++x) mbar_init(&bars[UNIT_EMPTY + x], 2 + kEpiWarps);
+        for (int x = 0; x < kUnitRing; ++x) mbar_init(&bars[UNIT_EMPTY + x], 2 + kEpiWarps);
         fence_mbar_init();
         *lut_valid = 1;
     }
@@ -563,11 +486,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             prefetch_tmap(&args.tv);
             prefetch_tmap(&args.tdy);
             prefetch_tmap(&args.tdyl);
-            UnitFeed un(p, bars, unit_slots, args.unit_ctr, args.nkt, 0);
+            UnitFeed<FEED_PRODUCER, true, BN> un(p, ring, args.nkt);
             int n = 0, g = 0;
             bool ok = true;
             while (ok && un.next()) {
-                const int row0 = (int)un.s.start, j0 = un.kt * BN;
+                const int row0 = (int)un.s.start, j0 = un.tile * BN;
                 if (n >= 1 && !mbar_wait(&bars[KV_EMPTY], (n - 1) & 1)) { ok = false; break; }
                 mbar_arrive_expect_tx(&bars[KV_FULL], L::KB + L::VB);
                 for (int kb = 0; kb < DQK / 64; ++kb)
@@ -611,12 +534,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t k_addr = sm_base + L::K_OFF, v_addr = sm_base + L::V_OFF;
             const uint32_t q_addr = sm_base + L::Q_OFF, y_addr = sm_base + L::Y_OFF;
             const uint32_t yl_addr = sm_base + L::YL_OFF, ds_addr = sm_base + L::YL_OFF;
-            UnitFeed un(p, bars, unit_slots, args.unit_ctr, args.nkt, 1);
+            UnitFeed<FEED_THREAD, true, BN> un(p, ring, args.nkt);
             int n = 0, g = 0;
             bool ok = true;
             while (ok && un.next()) {
                 if (!mbar_wait(&bars[KV_FULL], n & 1)) { ok = false; break; }
-                QTileIter t(un.s, un.kt * BN, p.W);
+                QTileIter t(un.s, un.tile * BN, p.W);
                 int x = 0;
                 while (t.next()) {
                     if (!mbar_wait(&bars[QD_FULL], g & 1)) { ok = false; break; }
@@ -690,12 +613,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 2) {
         // -------------------------------------------------------------------- query stamps
         const bool use_ts = p.NB > 0;
-        UnitFeed un(p, bars, unit_slots, args.unit_ctr, args.nkt, 2);
+        UnitFeed<FEED_WARP, true, BN> un(p, ring, args.nkt);
         int g = 0;
         bool ok = true;
         while (ok && un.next()) {
             const SeqInfo &s = un.s;
-            QTileIter t(s, un.kt * BN, p.W);
+            QTileIter t(s, un.tile * BN, p.W);
             while (t.next()) {
                 const int st = g & 1;
                 // the epilogue has finished with the stamps of tile g - 2
@@ -752,12 +675,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         e.lut = lut;
         e.tb_slot = tb_slot;
         e.d_rel = args.d_rel;
-        UnitFeed un(p, bars, unit_slots, args.unit_ctr, args.nkt, 2);
+        UnitFeed<FEED_WARP, true, BN> un(p, ring, args.nkt);
         int n = 0, g = 0;
         bool ok = true;
         while (ok && un.next()) {
             const SeqInfo &s = un.s;
-            const int j0 = un.kt * BN, jw = j0 + (warp & 3) * 32;
+            const int j0 = un.tile * BN, jw = j0 + (warp & 3) * 32;
             KeyLane k;
             k.j = j0 + r;
             k.key_in = k.j < s.L;

@@ -36,6 +36,7 @@
 #include "bias.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
+#include "units.cuh"
 
 namespace hstu {
 
@@ -57,7 +58,8 @@ constexpr float kTruncBump = 1.0028f;
 
 enum Bar { Q_FULL = 0, Q_EMPTY = 2, K_FULL = 4, K_EMPTY = 6, V_FULL = 8, V_EMPTY = 10,
            S_FULL = 12, S_FREE = 14, P_FULL = 16, P_FREE = 18, META_FULL = 20, EPI_DONE = 22,
-           O_FULL = 24, O_FREE = 25, MMA_DONE = 26, NUM_BARS = 27 };
+           O_FULL = 24, O_FREE = 25, MMA_DONE = 26, UNIT_FULL = 27, UNIT_EMPTY = 31,  // +4
+           NUM_BARS = 35 };
 
 struct TileMeta {
     int64_t tmin[4], tmax[4];   // timestamp range of each 32-key quarter (valid keys only)
@@ -73,8 +75,9 @@ struct FwdLayout {
     static constexpr int K_OFF = Q_OFF + QST * QB;
     static constexpr int V_OFF = K_OFF + KST * KB;
     static constexpr int BAR_OFF = V_OFF + VST * VB;
-    static constexpr int SLOT_OFF = BAR_OFF + 8 * 32;
-    static constexpr int META_OFF = SLOT_OFF + 16;
+    static constexpr int SLOT_OFF = BAR_OFF + 8 * 40;
+    static constexpr int UNIT_OFF = SLOT_OFF + 16;                 // kUnitRing unit indices
+    static constexpr int META_OFF = UNIT_OFF + 8 * kUnitRing;
     static constexpr int TSK_OFF = META_OFF + 2 * (int)sizeof(TileMeta);
     static constexpr int TSK32_OFF = TSK_OFF + 2 * BN * 8;
     static constexpr int LUT_OFF = TSK32_OFF + 2 * BN * 4;
@@ -89,6 +92,7 @@ struct FwdTcArgs {
     CUtensorMap tq, tk, tv;
     DevParams p;
     float *y;
+    unsigned long long *unit_ctr;   // next work unit to hand out (zeroed by the caller)
     int nqt;   // query tiles of the longest admissible sequence: ceil(N / 128)
 };
 
@@ -113,51 +117,11 @@ struct TileIter {
     }
 };
 
-// This CTA's work units, longest first: unit u = blockIdx.x + k * gridDim.x of the order
-// (query tile descending, then sequence, then head); units past a sequence's end are
-// skipped.  Every role walks the same sequence of units.
-struct UnitIter {
-    const DevParams &p;
-    int nqt;
-    int64_t u, total;
-    bool report;
-    SeqInfo s;
-    int qt, b, h;
-    __device__ UnitIter(const DevParams &p_, int nqt_, bool report_)
-        : p(p_), nqt(nqt_), u((int64_t)blockIdx.x - gridDim.x),
-          total((int64_t)nqt_ * p_.B * p_.H), report(report_) {}
-    __device__ bool next()
-    {
-        while ((u += gridDim.x) < total) {
-            const int64_t bh = (int64_t)p.B * p.H;
-            qt = nqt - 1 - (int)(u / bh);
-            const int rem = (int)(u % bh);
-            b = rem / p.H;
-            h = rem % p.H;
-            if (!seq_may_have_tile(p, b, qt)) continue;
-            s = load_seq(p, b, report && qt == 0 && h == 0);
-            if (qt * BM < s.L) return true;
-        }
-        return false;
-    }
-};
-
 __device__ __forceinline__ void report_timeout(const DevParams &p)
 {
     flag_error(p, HSTU_DEV_WAIT_TIMEOUT);
 }
 
-__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity)
-{
-    return __all_sync(0xffffffffu, mbar_wait(bar, parity));
-}
-
-// One arrival per warp on `bar` (counted per warp), after the whole warp got here.
-__device__ __forceinline__ void warp_arrive(uint64_t *bar)
-{
-    __syncwarp();
-    if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
-}
 
 // SPLIT: A enters A V as a pair of bf16 values, hi = bf16(A) and lo = bf16(A - hi), so Y
 // carries about 16 significant bits (used when Y is saved for the backward, whose
@@ -280,6 +244,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::BAR_OFF);
     uint32_t *slot = reinterpret_cast<uint32_t *>(sm + L::SLOT_OFF);
     int32_t *lut_valid = reinterpret_cast<int32_t *>(sm + L::SLOT_OFF + 4);
+    // Work units: query tiles from the last down (the longest rows first), sequence, head.
+    const FeedRing ring{bars + UNIT_FULL, bars + UNIT_EMPTY,
+                        reinterpret_cast<int64_t *>(sm + L::UNIT_OFF), args.unit_ctr};
     TileMeta *meta = reinterpret_cast<TileMeta *>(sm + L::META_OFF);
     int64_t *tsk = reinterpret_cast<int64_t *>(sm + L::TSK_OFF);
     int32_t *tsk32 = reinterpret_cast<int32_t *>(sm + L::TSK32_OFF);
@@ -298,6 +265,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             mbar_init(&bars[EPI_DONE + x], kEpiWarps);
         }
         mbar_init(&bars[O_FREE], kEpiWarps);
+        for (int x = 0; x < kUnitRing; ++x) mbar_init(&bars[UNIT_EMPTY + x], 3 + kEpiWarps);
         fence_mbar_init();
         *lut_valid = 1;
     }
@@ -326,11 +294,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             // ---------------------------------------------------------------- Q and K loads
             prefetch_tmap(&args.tq);
             prefetch_tmap(&args.tk);
-            UnitIter un(p, args.nqt, true);
+            UnitFeed<FEED_PRODUCER, false, BM> un(p, ring, args.nqt);
             int n = 0, g = 0;
             bool ok = true;
             while (ok && un.next()) {
-                const int i0 = un.qt * BM, row0 = (int)un.s.start, qs = n % QST;
+                const int i0 = un.tile * BM, row0 = (int)un.s.start, qs = n % QST;
                 if (n >= QST && !mbar_wait(&bars[Q_EMPTY + qs], (n / QST - 1) & 1)) {
                     ok = false;
                     break;
@@ -354,7 +322,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 }
                 ++n;
             }
-            if (!ok) report_timeout(p);
+            if (!ok || !un.ok) report_timeout(p);
             // loads issued must land before the CTA exits (bounded)
             bool drained = true;
             for (int x = n - 1; x >= 0 && x >= n - QST; --x)
@@ -367,12 +335,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (lane == 0) {
             // ---------------------------------------------------------------- V loads
             prefetch_tmap(&args.tv);
-            UnitIter un(p, args.nqt, false);
+            UnitFeed<FEED_THREAD, false, BM> un(p, ring, args.nqt);
             int g = 0;
             bool ok = true;
             while (ok && un.next()) {
                 const int row0 = (int)un.s.start;
-                TileIter t(un.s, un.qt * BM, p.W);
+                TileIter t(un.s, un.tile * BM, p.W);
                 while (t.next()) {
                     const int st = g % VST;
                     if (g >= VST && !mbar_wait(&bars[V_EMPTY + st], (g / VST - 1) & 1)) {
@@ -386,7 +354,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     ++g;
                 }
             }
-            if (!ok) report_timeout(p);
+            if (!ok || !un.ok) report_timeout(p);
             bool drained = true;
             for (int x = g - 1; x >= 0 && x >= g - VST; --x)
                 drained &= mbar_wait(&bars[V_FULL + x % VST], (x / VST) & 1);
@@ -422,7 +390,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 if (last) umma_commit(&bars[O_FULL]);
                 return true;
             };
-            UnitIter un(p, args.nqt, false);
+            UnitFeed<FEED_THREAD, false, BM> un(p, ring, args.nqt);
             int n = 0, g = 0;
             bool ok = true;
             bool pend = false;                  // an A V waiting for its A
@@ -433,7 +401,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 if (!mbar_wait(&bars[Q_FULL + qs], (n / QST) & 1)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t q_addr = sm_base + L::Q_OFF + qs * L::QB;
-                TileIter t(un.s, un.qt * BM, p.W);
+                TileIter t(un.s, un.tile * BM, p.W);
                 bool first = true, more = t.next();
                 while (more) {
                     const int st = g & 1, ks = g % KST;
@@ -468,7 +436,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 ++n;
             }
             if (ok && pend) ok = issue_pv(pg, pn, pfirst, true);
-            if (!ok) report_timeout(p);
+            if (!ok || !un.ok) report_timeout(p);
             // every MMA issued must complete before TMEM is released (bounded)
             umma_commit(&bars[MMA_DONE]);
             if (!mbar_wait(&bars[MMA_DONE], 0)) report_timeout(p);
@@ -476,12 +444,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     } else if (warp == 3) {
         // -------------------------------------------------------------------- tile metadata
         const bool use_ts = p.NB > 0;
-        UnitIter un(p, args.nqt, false);
+        UnitFeed<FEED_WARP, false, BM> un(p, ring, args.nqt);
         int g = 0;
         bool ok = true;
         while (ok && un.next()) {
             const SeqInfo &s = un.s;
-            TileIter t(s, un.qt * BM, p.W);
+            TileIter t(s, un.tile * BM, p.W);
             while (t.next()) {
                 const int st = g & 1;
                 // the epilogue is done with this stage's stamps (tile g - 2)
@@ -545,12 +513,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const float rel_sc = rel_in_smem ? 1.0f : tscale;  // relp * rel_sc = scaled half rel bias
         const float half_alpha = SPLIT ? 0.5f * p.alpha : 0.5f * kTruncBump * p.alpha;
         const bool lut_ok = *lut_valid != 0;
-        UnitIter un(p, args.nqt, false);
+        UnitFeed<FEED_WARP, false, BM> un(p, ring, args.nqt);
         int n = 0, g = 0;
         bool ok = true;
         while (ok && un.next()) {
             const SeqInfo &s = un.s;
-            const int i0 = un.qt * BM;
+            const int i0 = un.tile * BM;
             const int i = i0 + r;
             const bool row_in = i < s.L;
             const int pi = clamp_pos(i, s.E);
@@ -667,7 +635,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             }
             ++n;
         }
-        if (!ok) report_timeout(p);
+        if (!ok || !un.ok) report_timeout(p);
     }
 
     tc_fence_before();
@@ -751,12 +719,14 @@ bool tc_fwd_supported(int dqk, int dv, int64_t T)
 }
 
 cudaError_t launch_tc_fwd(const DevParams &p, const void *q, const void *k, const void *v,
-                          float *y, bool training, cudaStream_t st)
+                          float *y, unsigned long long *unit_ctr, bool training,
+                          cudaStream_t st)
 {
     FwdTcArgs a;
     std::memset(&a, 0, sizeof(a));
     a.p = p;
     a.y = y;
+    a.unit_ctr = unit_ctr;
     a.nqt = (p.N + BM - 1) / BM;
     if (!encode_tmap_bf16(&a.tq, q, p.dqk, p.H, p.T) || !encode_tmap_bf16(&a.tk, k, p.dqk, p.H, p.T) ||
         !encode_tmap_bf16(&a.tv, v, p.dv, p.H, p.T))

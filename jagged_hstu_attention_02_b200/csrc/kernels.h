@@ -71,8 +71,10 @@ cudaError_t launch_convert(const float *src, void *dst, int64_t n, cudaStream_t 
 // tcgen05 forward attention (bf16): Y = (1/N) sum_j A_ij V_j in fp32.  `training` selects
 // the variant whose Y carries ~16 significant bits (A split into bf16 hi + lo parts).
 bool tc_fwd_supported(int dqk, int dv, int64_t T);
+// unit_ctr: work-unit counter in device memory, zero at launch.
 cudaError_t launch_tc_fwd(const DevParams &p, const void *q, const void *k, const void *v,
-                          float *y, bool training, cudaStream_t st);
+                          float *y, unsigned long long *unit_ctr, bool training,
+                          cudaStream_t st);
 
 // Multiprocessors of the current device (cached after the first query).
 int num_sms();
