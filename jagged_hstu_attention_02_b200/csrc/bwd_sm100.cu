@@ -87,8 +87,8 @@ struct BwdLayout {
     static constexpr int YL_OFF = Y_OFF + YB;     // also DS
     static constexpr int BAR_OFF = YL_OFF + LB;
     static constexpr int SLOT_OFF = BAR_OFF + 8 * 32;
-    static constexpr int UNIT_OFF = SLOT_OFF + 16;                 // kUnitRing unit indices
-    static constexpr int META_OFF = UNIT_OFF + 8 * kUnitRing;
+    static constexpr int UNIT_OFF = SLOT_OFF + 16;                 // kUnitRing unit slots
+    static constexpr int META_OFF = UNIT_OFF + (int)sizeof(UnitSlot) * kUnitRing;
     static constexpr int TSQ_OFF = META_OFF + 2 * (int)sizeof(QMeta);
     static constexpr int TSQ32_OFF = TSQ_OFF + 2 * BM * 8;
     static constexpr int LUT_OFF = TSQ32_OFF + 2 * BM * 4;
@@ -428,7 +428,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int32_t *lut_valid = reinterpret_cast<int32_t *>(sm + L::SLOT_OFF + 4);
     // Work units: key tiles from the first up (the most query tiles first), sequence, head.
     const FeedRing ring{bars + UNIT_FULL, bars + UNIT_EMPTY,
-                        reinterpret_cast<int64_t *>(sm + L::UNIT_OFF), args.unit_ctr};
+                        reinterpret_cast<UnitSlot *>(sm + L::UNIT_OFF), args.unit_ctr};
     QMeta *meta = reinterpret_cast<QMeta *>(sm + L::META_OFF);
     int64_t *tsq = reinterpret_cast<int64_t *>(sm + L::TSQ_OFF);
     int32_t *tsq32 = reinterpret_cast<int32_t *>(sm + L::TSQ32_OFF);

@@ -76,8 +76,8 @@ struct FwdLayout {
     static constexpr int V_OFF = K_OFF + KST * KB;
     static constexpr int BAR_OFF = V_OFF + VST * VB;
     static constexpr int SLOT_OFF = BAR_OFF + 8 * 40;
-    static constexpr int UNIT_OFF = SLOT_OFF + 16;                 // kUnitRing unit indices
-    static constexpr int META_OFF = UNIT_OFF + 8 * kUnitRing;
+    static constexpr int UNIT_OFF = SLOT_OFF + 16;                 // kUnitRing unit slots
+    static constexpr int META_OFF = UNIT_OFF + (int)sizeof(UnitSlot) * kUnitRing;
     static constexpr int TSK_OFF = META_OFF + 2 * (int)sizeof(TileMeta);
     static constexpr int TSK32_OFF = TSK_OFF + 2 * BN * 8;
     static constexpr int LUT_OFF = TSK32_OFF + 2 * BN * 4;
@@ -246,7 +246,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     int32_t *lut_valid = reinterpret_cast<int32_t *>(sm + L::SLOT_OFF + 4);
     // Work units: query tiles from the last down (the longest rows first), sequence, head.
     const FeedRing ring{bars + UNIT_FULL, bars + UNIT_EMPTY,
-                        reinterpret_cast<int64_t *>(sm + L::UNIT_OFF), args.unit_ctr};
+                        reinterpret_cast<UnitSlot *>(sm + L::UNIT_OFF), args.unit_ctr};
     TileMeta *meta = reinterpret_cast<TileMeta *>(sm + L::META_OFF);
     int64_t *tsk = reinterpret_cast<int64_t *>(sm + L::TSK_OFF);
     int32_t *tsk32 = reinterpret_cast<int32_t *>(sm + L::TSK32_OFF);

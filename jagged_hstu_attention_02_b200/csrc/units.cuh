@@ -33,10 +33,17 @@ __device__ __forceinline__ void warp_arrive(uint64_t *bar)
 
 enum FeedRole { FEED_PRODUCER, FEED_THREAD, FEED_WARP };
 
+// One published unit: its number (-1: no more units) and its sequence, read once by the
+// producer so that consumers start the unit without global loads.
+struct UnitSlot {
+    int64_t u;
+    SeqInfo s;
+};
+
 // The shared-memory ring and the global counter of one CTA.
 struct FeedRing {
     uint64_t *full, *empty;      // kUnitRing barriers each
-    int64_t *slots;              // kUnitRing unit numbers
+    UnitSlot *slots;             // kUnitRing slots
     unsigned long long *ctr;
 };
 
@@ -49,7 +56,7 @@ template <int ROLE, bool ASCENDING, int TILE>
 struct UnitFeed {
     const DevParams &p;
     uint64_t *full, *empty;
-    int64_t *slots;
+    UnitSlot *slots;
     unsigned long long *ctr;
     int ntiles;
     int64_t total;
@@ -106,7 +113,8 @@ struct UnitFeed {
                 ok = false;
                 return false;
             }
-            slots[sl] = u;
+            slots[sl].u = u;
+            if (u >= 0) slots[sl].s = s;
             mbar_arrive(&full[sl]);      // releases the slot's contents
             return u >= 0;
         } else {
@@ -116,12 +124,12 @@ struct UnitFeed {
                 ok = false;
                 return false;
             }
-            const int64_t u = *reinterpret_cast<volatile int64_t *>(&slots[sl]);
+            const int64_t u = slots[sl].u;
+            if (u >= 0) s = slots[sl].s;
             if constexpr (ROLE == FEED_WARP) warp_arrive(&empty[sl]);
             else mbar_arrive(&empty[sl]);
             if (u < 0) return false;
             decode(u);
-            s = load_seq(p, b, false);
             return true;
         }
     }
