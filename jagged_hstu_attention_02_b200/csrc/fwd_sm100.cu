@@ -158,35 +158,41 @@ __device__ __forceinline__ void fwd_quarter(const FwdEpi &e, const HalfTime &ht,
     const uint32_t a1 = (uint32_t)ht.cmpA + 1u;
     const int64_t sp = (int64_t)ht.cmpB - (int64_t)ht.cmpA - 1;
     const uint32_t span = sp > 0 ? (uint32_t)sp : 0u;
+    const float2 ha2 = make_float2(e.half_alpha, e.half_alpha);
+    const float2 rs2 = make_float2(e.rel_sc, e.rel_sc);
 #pragma unroll 1   // one copy of the 8-key body per mode combination (instruction cache)
     for (int ch = 0; ch < 4; ++ch) {
         const int cb = ch * 8;
         uint32_t ra[8];
-        tmem_ld8(e.t_s + cb, ra);
-        tmem_wait_ld();
-        reg_fence(ra);
-        float bh[8];   // half of the bias
+        tmem_ld8(e.t_s + cb, ra);   // S arrives while the bias, which does not need it, is formed
+        float tb[8], rv[8];
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
-            float tb;
             if (TM == 0) {
-                tb = ht.tb_lo;
+                tb[c] = ht.tb_lo;
             } else if (TM == 1) {
                 const bool lo = (uint32_t)e.tk32[cb + c] - a1 < span;
-                tb = lo ? ht.tb_lo : ht.tb_hi;
+                tb[c] = lo ? ht.tb_lo : ht.tb_hi;
             } else if (TM == 2) {
                 const int32_t d = ht.t_rel - e.tk32[cb + c];
                 uint32_t dt = (uint32_t)(d < 0 ? -d : d);
                 dt = min(dt, (uint32_t)INT32_MAX - 1u);
                 const float v = e.tbh[lut_bucket(e.lut, dt)];
-                tb = ht.lane_const ? ht.tb_lo : v;
+                tb[c] = ht.lane_const ? ht.tb_lo : v;
             } else {
-                tb = e.tbh[bucket_search(e.thr, e.n_thr, abs_diff_u64(e.tsi, e.tk64[cb + c]))];
+                tb[c] = e.tbh[bucket_search(e.thr, e.n_thr, abs_diff_u64(e.tsi, e.tk64[cb + c]))];
             }
             int ri = e.rbase - cb - c;
             if (!RD) ri = ri < 0 ? 0 : (ri > e.R - 1 ? e.R - 1 : ri);
-            bh[c] = fmaf(e.relp[ri], e.rel_sc, tb);
+            rv[c] = e.relp[ri];
         }
+        float2 bh[4];   // half of the bias, key pairs
+#pragma unroll
+        for (int c2 = 0; c2 < 4; ++c2)
+            bh[c2] = __ffma2_rn(make_float2(rv[2 * c2], rv[2 * c2 + 1]), rs2,
+                                make_float2(tb[2 * c2], tb[2 * c2 + 1]));
+        tmem_wait_ld();
+        reg_fence(ra);
         // SiLU(x) = x sigmoid(x) = h + h tanh(h), h = x/2; mask after the nonlinearity
         const uint32_t vb = vmask >> cb;
         uint32_t pk[4];
@@ -195,11 +201,15 @@ __device__ __forceinline__ void fwd_quarter(const FwdEpi &e, const HalfTime &ht,
             uint32_t plo[4];
 #pragma unroll
             for (int c2 = 0; c2 < 4; ++c2) {
+                // h = x/2 (exact halving: x = 2h is alpha s + bias with one rounding)
+                const float2 h = __ffma2_rn(ha2, make_float2(__uint_as_float(ra[2 * c2]),
+                                                             __uint_as_float(ra[2 * c2 + 1])),
+                                            bh[c2]);
                 float a[2];
 #pragma unroll
                 for (int q = 0; q < 2; ++q) {
                     const int c = 2 * c2 + q;
-                    const float xs = fmaf(e.alpha, __uint_as_float(ra[c]), 2.0f * bh[c]);
+                    const float xs = 2.0f * (q ? h.y : h.x);
                     const float v = xs * __fdividef(1.0f, 1.0f + __expf(-xs));
                     a[q] = (FULL || ((vb >> c) & 1u)) ? v : 0.f;
                 }
@@ -214,10 +224,11 @@ __device__ __forceinline__ void fwd_quarter(const FwdEpi &e, const HalfTime &ht,
             // (A is rounded to bf16 for the tensor core either way)
 #pragma unroll
             for (int c2 = 0; c2 < 4; ++c2) {
-                const float x0 = fmaf(e.half_alpha, __uint_as_float(ra[2 * c2]), bh[2 * c2]);
-                const float x1 = fmaf(e.half_alpha, __uint_as_float(ra[2 * c2 + 1]), bh[2 * c2 + 1]);
-                // bf16 pair = the high halves of x0, x1 (one byte permute)
-                const uint32_t h2 = __byte_perm(__float_as_uint(x0), __float_as_uint(x1), 0x7632);
+                const float2 x = __ffma2_rn(ha2, make_float2(__uint_as_float(ra[2 * c2]),
+                                                             __uint_as_float(ra[2 * c2 + 1])),
+                                            bh[c2]);
+                // bf16 pair = the high halves of x.x, x.y (one byte permute)
+                const uint32_t h2 = __byte_perm(__float_as_uint(x.x), __float_as_uint(x.y), 0x7632);
                 uint32_t a2 = fma_bf16x2(h2, tanh_bf16x2(h2), h2);
                 if (!FULL)
                     a2 &= (((vb >> (2 * c2)) & 1u) ? 0x0000FFFFu : 0u) |
