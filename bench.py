@@ -180,14 +180,14 @@ def run_ours(args, world, rank, local):
     ws_b = ops.bwd.last_workspace
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
 
-    def step():
+    def step(collective=True):
         ops.fwd(dev["q"], dev["k"], dev["v"], dev["u"], dev["seq_offsets"],
                 dev["num_contextuals"], dev["num_targets"], dev["timestamps"], dev["rel_bias"],
                 dev["time_bias"], training=True, out=out, saved=saved, workspace=ws_f, **kw)
         ops.bwd(dev["dout"], dev["q"], dev["k"], dev["v"], dev["u"], dev["seq_offsets"],
                 dev["num_contextuals"], dev["num_targets"], dev["timestamps"], dev["rel_bias"],
                 dev["time_bias"], saved=saved, grads=grads, workspace=ws_b, **kw)
-        if world > 1:
+        if world > 1 and collective:
             torch.distributed.all_reduce(table_grads)
 
     stages = ["fwd_attn", "fwd_norm", "bwd_norm", "bwd_attn"]
@@ -195,9 +195,41 @@ def run_ours(args, world, rank, local):
         flush.fill_(1.0)
         step()
     torch.cuda.synchronize()
+    # per-stage times of eager steps (events between every kernel, so each includes its
+    # launch gap); they pick the dominant kernel, the one timed inside the measured steps
     evs = stage_timer(ops, torch, stages)
     stage_ms = {s: [] for s in stages}
-    step_ms = []
+    for _ in range(max(3, args.warmup)):
+        flush.fill_(1.0)
+        step()
+        torch.cuda.synchronize()
+        for s in stages:
+            stage_ms[s].append(evs[s][0].elapsed_time(evs[s][1]))
+    for s in stages:
+        ops.set_stage_events(s)
+    avg = {s: sum(v) / len(v) for s, v in stage_ms.items()}
+    dom = max(avg, key=avg.get)
+    dom_ev = stage_timer(ops, torch, [dom])[dom]
+
+    # the measured steps replay one CUDA graph of the step's library calls (the table-grad
+    # all-reduce of a sharded step stays outside it); only the dominant kernel's two events
+    # are recorded inside
+    graph = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream()
+    cap.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(cap):
+        with torch.cuda.graph(graph, stream=cap):
+            step(collective=False)
+    torch.cuda.current_stream().wait_stream(cap)
+    torch.cuda.synchronize()
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        graph.replay()
+        if world > 1:
+            torch.distributed.all_reduce(table_grads)
+    torch.cuda.synchronize()
+
+    step_ms, dom_ms = [], []
     clocks = ClockSampler(local)
     clocks.start()
     if world > 1:
@@ -208,20 +240,21 @@ def run_ours(args, world, rank, local):
         flush.fill_(1.0)                       # evict the previous step's data from L2
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
-        step()
+        graph.replay()
+        if world > 1:
+            torch.distributed.all_reduce(table_grads)
         e1.record()
         e1.synchronize()
         step_ms.append(e0.elapsed_time(e1))
-        for s in stages:
-            stage_ms[s].append(evs[s][0].elapsed_time(evs[s][1]))
+        dom_ms.append(dom_ev[0].elapsed_time(dom_ev[1]))
     torch.cuda.synchronize()
     wall_region = time.perf_counter() - t_region
     if world > 1:
         torch.distributed.barrier()
     clk = clocks.stop()
-    for s in stages:
-        ops.set_stage_events(s)
+    ops.set_stage_events(dom)
     assert ops.read_device_status(ws_f) == 0 and ops.read_device_status(ws_b) == 0
+    del graph
 
     ms = sum(step_ms) / len(step_ms)
     if world > 1:
@@ -230,9 +263,8 @@ def run_ours(args, world, rank, local):
         ms = float(t.item())
     value = world * flops / (ms * 1e-3) / 1e12
 
-    # roofline of the dominant kernel stage
-    avg = {s: sum(v) / len(v) for s, v in stage_ms.items()}
-    dom = max(avg, key=avg.get)
+    # roofline of the dominant kernel stage, timed inside the measured steps
+    avg[dom] = sum(dom_ms) / len(dom_ms)
     dom_bytes = {"fwd_attn": accounting.fwd_bytes(b, training=True),
                  "fwd_norm": b.total_tokens * b.num_heads * b.d_v * (4 + 2 + 2) + 8 * tokens,
                  "bwd_norm": b.total_tokens * b.num_heads * b.d_v * (2 + 2 + 4 + 2 + 4) + 8 * tokens,
@@ -245,7 +277,9 @@ def run_ours(args, world, rank, local):
                 "unit": "GB/s", "frac": round(achieved / hbm_peak, 4), "traffic": traffic,
                 "traffic_note": traffic_note, "algorithmic_bytes": dom_bytes,
                 "kernel_stage": dom, "kernel_ms": round(avg[dom], 4),
-                "peak_source": peak_kind, "stage_ms": {s: round(v, 4) for s, v in avg.items()}}
+                "peak_source": peak_kind, "stage_ms": {s: round(v, 4) for s, v in avg.items()},
+                "stage_ms_note": "kernel_ms timed inside the measured graph replays; the other "
+                                 "stages from eager steps with events between all kernels"}
     if dom in dom_flops:
         roofline["tflops"] = round(dom_flops[dom] / (avg[dom] * 1e-3) / 1e12, 2)
 
@@ -270,6 +304,7 @@ def run_ours(args, world, rank, local):
                    "tokens_per_gpu": tokens, "valid_pairs_per_gpu": P, "flops_per_step": flops,
                    "max_seqlen": b.max_seqlen, "parallelism": "dp%d" % world,
                    "l2": "flushed between steps (256 MB write), flush outside per-step events",
+                   "launch": "each step replays one CUDA graph of its fwd and bwd library calls",
                    "wall_s_region": round(wall_region, 3)},
         "roofline": roofline, "e2e": e2e, "clocks": clk,
         "gpu_launches": args.steps * LAUNCHES_PER_STEP,

@@ -195,7 +195,9 @@ hstu_status_t hstu_attn_fwd_noalloc(const hstu_attn_params_t *params, const void
 /*
  * Measurement hook.  While set, every fwd/bwd call records `start_event` on its stream just
  * before launching the kernel(s) of `stage` and `stop_event` just after (both cudaEvent_t).
- * NULL events clear the hook.  Process-wide and not thread-safe: for benchmarks only.
+ * NULL events clear the hook.  Process-wide and not thread-safe: for benchmarks only.  A
+ * call made while its stream is being captured into a CUDA graph records the events as
+ * graph nodes of their own, so every replay of the graph stamps them.
  */
 hstu_status_t hstu_attn_set_stage_events(int32_t stage, void *start_event, void *stop_event);
 

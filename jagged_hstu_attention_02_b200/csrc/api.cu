@@ -136,16 +136,27 @@ size_t bwd_ws_bytes(const hstu_attn_params_t *p)
 
 cudaEvent_t g_stage_ev[HSTU_NUM_STAGES][2];
 
+// Records an event on s.  Inside a stream capture the record becomes a graph node of its
+// own (external), so that each replay of the graph stamps the event.
+void record_stage_event(cudaEvent_t e, cudaStream_t s)
+{
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusActive)
+        cudaEventRecordWithFlags(e, s, cudaEventRecordExternal);
+    else
+        cudaEventRecord(e, s);
+}
+
 struct StageScope {
     int stage;
     cudaStream_t s;
     StageScope(int st, cudaStream_t str) : stage(st), s(str)
     {
-        if (g_stage_ev[stage][0]) cudaEventRecord(g_stage_ev[stage][0], s);
+        if (g_stage_ev[stage][0]) record_stage_event(g_stage_ev[stage][0], s);
     }
     ~StageScope()
     {
-        if (g_stage_ev[stage][1]) cudaEventRecord(g_stage_ev[stage][1], s);
+        if (g_stage_ev[stage][1]) record_stage_event(g_stage_ev[stage][1], s);
     }
 };
 
