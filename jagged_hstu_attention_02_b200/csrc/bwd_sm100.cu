@@ -241,8 +241,46 @@ __device__ __forceinline__ void epi_block(const DevParams &p, const EpiBlock &e,
     for (int ch = 0; ch < 4; ++ch) {
         // 8 query columns: one 16-byte chunk of the dS^T row, 4 TMEM columns of A^T
         uint32_t rs[8], rd[8];
-        tmem_ld8(e.t_s + ch * 8, rs);
+        tmem_ld8(e.t_s + ch * 8, rs);   // S and dP arrive while the biases are formed
         tmem_ld8(e.t_dp + ch * 8, rd);
+        float bias[8];
+        int bkv[8], riv[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const int cc = ch * 8 + c;
+            const int i = e.iq + cc;
+            int bk = 0;
+            if (TM == 0) {
+                bias[c] = ht.tb_lo;
+            } else if (TM == 1) {
+                const int32_t t = e.tq32[cc];
+                const bool hi = t <= ht.cmpA || t >= ht.cmpB;
+                bias[c] = hi ? ht.tb_hi : ht.tb_lo;
+                bk = hi ? 1 : 0;
+            } else if (TM == 2) {
+                const int32_t d = ht.t_rel - e.tq32[cc];
+                uint32_t dt = (uint32_t)(d < 0 ? -d : d);
+                dt = min(dt, (uint32_t)INT32_MAX - 1u);
+                const int b = lut_bucket(e.lut, dt);
+                bk = ht.lane_const ? ht.blo : b;
+                bias[c] = ht.lane_const ? ht.tb_lo : e.tbs[b];
+            } else {
+                bk = bucket_search(e.thr, p.n_thr, abs_diff_u64(k.tsj, e.tq64[cc]));
+                bias[c] = e.tbs[bk];
+            }
+            int ri;
+            if (KIND == 0) {
+                ri = e.rbase + cc;
+            } else if (KIND == 1) {
+                ri = cc >= e.fc ? e.rc : e.rbase + cc;
+            } else {
+                const int rraw = min(i, e.Em1) - k.pj;
+                ri = rraw < 0 ? 0 : (rraw > p.R - 1 ? p.R - 1 : rraw);
+            }
+            bias[c] += e.relp[ri];
+            bkv[c] = bk;
+            riv[c] = ri;
+        }
         tmem_wait_ld();
         reg_fence(rs);
         reg_fence(rd);
@@ -255,43 +293,13 @@ __device__ __forceinline__ void epi_block(const DevParams &p, const EpiBlock &e,
 #pragma unroll
             for (int q = 0; q < 2; ++q) {
                 const int c = 2 * c2 + q, cc = ch * 8 + c;
-                const int i = e.iq + cc;
                 const bool valid = (e.vbits >> cc) & 1u;
-                // ---- bias
-                float bias;
-                int bk = 0;
-                if (TM == 0) {
-                    bias = ht.tb_lo;
-                } else if (TM == 1) {
-                    const int32_t t = e.tq32[cc];
-                    const bool hi = t <= ht.cmpA || t >= ht.cmpB;
-                    bias = hi ? ht.tb_hi : ht.tb_lo;
-                    bk = hi ? 1 : 0;
-                } else if (TM == 2) {
-                    const int32_t d = ht.t_rel - e.tq32[cc];
-                    uint32_t dt = (uint32_t)(d < 0 ? -d : d);
-                    dt = min(dt, (uint32_t)INT32_MAX - 1u);
-                    const int b = lut_bucket(e.lut, dt);
-                    bk = ht.lane_const ? ht.blo : b;
-                    bias = ht.lane_const ? ht.tb_lo : e.tbs[b];
-                } else {
-                    bk = bucket_search(e.thr, p.n_thr, abs_diff_u64(k.tsj, e.tq64[cc]));
-                    bias = e.tbs[bk];
-                }
-                int ri;
-                if (KIND == 0) {
-                    ri = e.rbase + cc;
-                } else if (KIND == 1) {
-                    ri = cc >= e.fc ? e.rc : e.rbase + cc;
-                } else {
-                    const int rraw = min(i, e.Em1) - k.pj;
-                    ri = rraw < 0 ? 0 : (rraw > p.R - 1 ? p.R - 1 : rraw);
-                }
-                bias += e.relp[ri];
+                const int bk = bkv[c], ri = riv[c];
+                const float bias_c = bias[c];
                 // ---- s = alpha q.k + b; SiLU(s) = s sigma(s); SiLU'(s) = sigma (1 + s (1 - sigma)).
                 // sigma from the accurate exponential: table gradients sum dS over many pairs
                 // and can cancel, so dS needs close to fp32 accuracy
-                const float xs = fmaf(p.alpha, __uint_as_float(rs[c]), bias);
+                const float xs = fmaf(p.alpha, __uint_as_float(rs[c]), bias_c);
                 const float sig = __fdividef(1.0f, 1.0f + __expf(-xs));
                 const float silu = xs * sig;
                 const float dsilu = sig * fmaf(xs, 1.0f - sig, 1.0f);
