@@ -480,6 +480,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     __threadfence();   // the zeroed slot row is in place before any reduction into it
     __syncthreads();
     if (p.NB > 0) build_lut(thr, p.n_thr, lut, lut_valid);
+    // the set-up above reads inputs only; dY and the zeroed accumulators come from the
+    // LayerNorm backward ahead on the stream
+    grid_dep_wait();
+    grid_dep_release();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -884,8 +888,7 @@ cudaError_t launch_bwd(const BwdTcArgs &a, cudaStream_t st)
     if (grid > kBwdMaxCtas) grid = kBwdMaxCtas;
     if (units < grid) grid = (int)units;
     if (grid <= 0) return cudaSuccess;
-    kern<<<grid, kThreads, L::ALLOC, st>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(kern, dim3(grid), dim3(kThreads), L::ALLOC, st, a);
 }
 
 }  // namespace

@@ -95,6 +95,20 @@ __device__ __forceinline__ bool seq_may_have_tile(const DevParams &p, int b, int
     return t < n || n == 255;
 }
 
+// Programmatic dependent launch.  A kernel started with launch_pdl may begin (its set-up:
+// tables, shared memory, TMEM) while the kernel ahead of it on the stream is still running.
+// grid_dep_wait() blocks until that kernel has completed and its writes are visible (a no-op
+// for a normal launch); grid_dep_release() lets the kernel behind this one start early.
+__device__ __forceinline__ void grid_dep_wait()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+__device__ __forceinline__ void grid_dep_release()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Transposes 16-byte chunks within groups of NCH lanes: on entry lane l holds chunks
 // 0..NCH-1 of row l; on exit lane l, j = l % NCH, holds chunk j of rows l - j .. l - j +
 // NCH-1 (slot c = row l - j + c).  Lets the NCH lanes of a group write one row's NCH

@@ -294,6 +294,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     fill_seq_tiles(p, kTcThreads);
     __syncthreads();
     if (p.NB > 0) build_lut(thr, p.n_thr, lutp, lut_valid);
+    grid_dep_release();   // the LayerNorm behind this kernel may be scheduled
     tc_fence_before();
     __syncthreads();
     tc_fence_after();

@@ -9,6 +9,26 @@
 
 namespace hstu {
 
+// Launches kern with programmatic stream serialisation: it may start while the kernel ahead
+// of it on the stream finishes, and must call grid_dep_wait() before it touches anything that
+// kernel writes or reads.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 template <typename T>
 cudaError_t launch_simt_fwd(const DevParams &p, const void *q, const void *k, const void *v,
                             float *y, cudaStream_t st);

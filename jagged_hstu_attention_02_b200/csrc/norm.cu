@@ -58,6 +58,7 @@ __global__ void __launch_bounds__(32 * kRows)
                        float *__restrict__ rstd_out)
 {
     using V = Vec4<T>;
+    grid_dep_wait();   // y comes from the attention kernel ahead on the stream
     const int lane = threadIdx.x & 31;
     const int64_t row = (int64_t)blockIdx.x * kRows + (threadIdx.x >> 5);
     if (row >= p.T) return;
@@ -109,6 +110,7 @@ __global__ void __launch_bounds__(32 * kRows)
                            T *__restrict__ du, DYT *__restrict__ dy, const BwdZero zj)
 {
     using V = Vec4<T>;
+    grid_dep_release();   // the attention backward may start its set-up
     const int lane = threadIdx.x & 31;
     const int64_t row = (int64_t)blockIdx.x * kRows + (threadIdx.x >> 5);
     bwd_zero_small(zj);
@@ -169,9 +171,8 @@ cudaError_t fwd_nv(const DevParams &p, const float *y, const void *u, void *out,
                    float *rstd, cudaStream_t st)
 {
     const int64_t blocks = (p.T + kRows - 1) / kRows;
-    ln_gate_vec_kernel<T, NV><<<(unsigned)blocks, 32 * kRows, 0, st>>>(
-        p, y, (const T *)u, (T *)out, mean, rstd);
-    return cudaGetLastError();
+    return launch_pdl(ln_gate_vec_kernel<T, NV>, dim3((unsigned)blocks), dim3(32 * kRows), 0, st,
+                      p, y, (const T *)u, (T *)out, mean, rstd);
 }
 
 template <typename T, int NV>

@@ -474,6 +474,7 @@ __global__ void __launch_bounds__(kThreads)
 template <typename T>
 __global__ void convert_kernel(const float *__restrict__ src, T *__restrict__ dst, int64_t n)
 {
+    grid_dep_wait();   // src is complete once the kernel ahead on the stream is
     for (int64_t x = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; x < n;
          x += (int64_t)gridDim.x * blockDim.x)
         dst[x] = from_f32<T>(src[x]);
@@ -546,8 +547,8 @@ cudaError_t launch_convert(const float *src, void *dst, int64_t n, cudaStream_t 
     if (n <= 0) return cudaSuccess;
     int64_t blocks = (n + 255) / 256;
     if (blocks > 148 * 16) blocks = 148 * 16;
-    convert_kernel<T><<<(unsigned)blocks, 256, 0, st>>>(src, (T *)dst, n);
-    return cudaGetLastError();
+    return launch_pdl(convert_kernel<T>, dim3((unsigned)blocks), dim3(256), 0, st, src, (T *)dst,
+                      n);
 }
 
 template cudaError_t launch_simt_fwd<float>(const DevParams &, const void *, const void *,
