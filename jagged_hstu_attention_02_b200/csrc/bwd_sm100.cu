@@ -238,16 +238,16 @@ __device__ __forceinline__ void epi_block(const DevParams &p, const EpiBlock &e,
     const bool lane0 = lane == 0;
     const int src = (lane + 31) & 31;
 #pragma unroll 1
-    for (int ch = 0; ch < 4; ++ch) {
-        // 8 query columns: one 16-byte chunk of the dS^T row, 4 TMEM columns of A^T
-        uint32_t rs[8], rd[8];
-        tmem_ld8(e.t_s + ch * 8, rs);   // S and dP arrive while the biases are formed
-        tmem_ld8(e.t_dp + ch * 8, rd);
-        float bias[8];
-        int bkv[8], riv[8];
+    for (int ch = 0; ch < 8; ++ch) {
+        // 4 query columns: half a 16-byte chunk of the dS^T row, 2 TMEM columns of A^T
+        uint32_t rs[4], rd[4];
+        tmem_ld4(e.t_s + ch * 4, rs);   // S and dP arrive while the biases are formed
+        tmem_ld4(e.t_dp + ch * 4, rd);
+        float bias[4];
+        int bkv[4], riv[4];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            const int cc = ch * 8 + c;
+        for (int c = 0; c < 4; ++c) {
+            const int cc = ch * 4 + c;
             const int i = e.iq + cc;
             int bk = 0;
             if (TM == 0) {
@@ -284,15 +284,15 @@ __device__ __forceinline__ void epi_block(const DevParams &p, const EpiBlock &e,
         tmem_wait_ld();
         reg_fence(rs);
         reg_fence(rd);
-        uint32_t pa[4], pd[4];
-        int tbk[8];        // TM >= 2: bucket of each pair (-1: masked) and its dS
-        float tds[8];
+        uint32_t pa[2], pd[2];
+        int tbk[4];        // TM >= 2: bucket of each pair (-1: masked) and its dS
+        float tds[4];
 #pragma unroll
-        for (int c2 = 0; c2 < 4; ++c2) {
+        for (int c2 = 0; c2 < 2; ++c2) {
             float av[2], dv2[2];
 #pragma unroll
             for (int q = 0; q < 2; ++q) {
-                const int c = 2 * c2 + q, cc = ch * 8 + c;
+                const int c = 2 * c2 + q, cc = ch * 4 + c;
                 const bool valid = (e.vbits >> cc) & 1u;
                 const int bk = bkv[c], ri = riv[c];
                 const float bias_c = bias[c];
@@ -342,15 +342,16 @@ __device__ __forceinline__ void epi_block(const DevParams &p, const EpiBlock &e,
             // runs of equal buckets over the chunk's pairs, after all of its loads: a flush
             // (inline asm) inside the pair loop would hold the next pairs' loads behind it
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
+            for (int c = 0; c < 4; ++c) {
                 const bool chg = tbk[c] >= 0 && tbk[c] != k.cur_b;
                 red_add_if(e.tb_slot + k.cur_b, k.run, chg && e.use_ts);
                 k.cur_b = chg ? tbk[c] : k.cur_b;
                 k.run = (chg ? 0.f : k.run) + tds[c];
             }
         }
-        tmem_st4(e.t_s + ch * 4, pa);
-        st_shared_v4(e.ds_row + (((e.ds_chunk0 + ch) ^ e.rsw) << 4), pd[0], pd[1], pd[2], pd[3]);
+        tmem_st2(e.t_s + ch * 2, pa);
+        st_shared_v2(e.ds_row + (((e.ds_chunk0 + (ch >> 1)) ^ e.rsw) << 4) + (ch & 1) * 8, pd[0],
+                     pd[1]);
     }
 }
 

@@ -160,14 +160,14 @@ __device__ __forceinline__ void fwd_quarter(const FwdEpi &e, const HalfTime &ht,
     const uint32_t span = sp > 0 ? (uint32_t)sp : 0u;
     const float2 ha2 = make_float2(e.half_alpha, e.half_alpha);
     const float2 rs2 = make_float2(e.rel_sc, e.rel_sc);
-#pragma unroll 1   // one copy of the 8-key body per mode combination (instruction cache)
-    for (int ch = 0; ch < 4; ++ch) {
-        const int cb = ch * 8;
-        uint32_t ra[8];
-        tmem_ld8(e.t_s + cb, ra);   // S arrives while the bias, which does not need it, is formed
-        float tb[8], rv[8];
+#pragma unroll 1   // one copy of the 4-key body per mode combination (instruction cache)
+    for (int ch = 0; ch < 8; ++ch) {
+        const int cb = ch * 4;
+        uint32_t ra[4];
+        tmem_ld4(e.t_s + cb, ra);
+        float tb[4], rv[4];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
+        for (int c = 0; c < 4; ++c) {
             if (TM == 0) {
                 tb[c] = ht.tb_lo;
             } else if (TM == 1) {
@@ -186,22 +186,19 @@ __device__ __forceinline__ void fwd_quarter(const FwdEpi &e, const HalfTime &ht,
             if (!RD) ri = ri < 0 ? 0 : (ri > e.R - 1 ? e.R - 1 : ri);
             rv[c] = e.relp[ri];
         }
-        float2 bh[4];   // half of the bias, key pairs
+        float2 bh[2];
 #pragma unroll
-        for (int c2 = 0; c2 < 4; ++c2)
+        for (int c2 = 0; c2 < 2; ++c2)
             bh[c2] = __ffma2_rn(make_float2(rv[2 * c2], rv[2 * c2 + 1]), rs2,
                                 make_float2(tb[2 * c2], tb[2 * c2 + 1]));
         tmem_wait_ld();
         reg_fence(ra);
-        // SiLU(x) = x sigmoid(x) = h + h tanh(h), h = x/2; mask after the nonlinearity
         const uint32_t vb = vmask >> cb;
-        uint32_t pk[4];
+        uint32_t pk[2];
         if constexpr (SPLIT) {
-            // training forward: accurate sigmoid in fp32, A split into hi + lo
-            uint32_t plo[4];
+            uint32_t plo[2];
 #pragma unroll
-            for (int c2 = 0; c2 < 4; ++c2) {
-                // h = x/2 (exact halving: x = 2h is alpha s + bias with one rounding)
+            for (int c2 = 0; c2 < 2; ++c2) {
                 const float2 h = __ffma2_rn(ha2, make_float2(__uint_as_float(ra[2 * c2]),
                                                              __uint_as_float(ra[2 * c2 + 1])),
                                             bh[c2]);
@@ -217,17 +214,14 @@ __device__ __forceinline__ void fwd_quarter(const FwdEpi &e, const HalfTime &ht,
                 plo[c2] = pack_bf16x2(a[0] - __uint_as_float(pk[c2] << 16),
                                       a[1] - __uint_as_float(pk[c2] & 0xFFFF0000u));
             }
-            tmem_st4(e.t_a + ch * 4, pk);
-            tmem_st4(e.t_a + 16 + ch * 4, plo);
+            tmem_st2(e.t_a + ch * 2, pk);
+            tmem_st2(e.t_a + 16 + ch * 2, plo);
         } else {
-            // inference forward: h in fp32, then tanh and h + h tanh(h) on bf16 pairs
-            // (A is rounded to bf16 for the tensor core either way)
 #pragma unroll
-            for (int c2 = 0; c2 < 4; ++c2) {
+            for (int c2 = 0; c2 < 2; ++c2) {
                 const float2 x = __ffma2_rn(ha2, make_float2(__uint_as_float(ra[2 * c2]),
                                                              __uint_as_float(ra[2 * c2 + 1])),
                                             bh[c2]);
-                // bf16 pair = the high halves of x.x, x.y (one byte permute)
                 const uint32_t h2 = __byte_perm(__float_as_uint(x.x), __float_as_uint(x.y), 0x7632);
                 uint32_t a2 = fma_bf16x2(h2, tanh_bf16x2(h2), h2);
                 if (!FULL)
@@ -235,7 +229,7 @@ __device__ __forceinline__ void fwd_quarter(const FwdEpi &e, const HalfTime &ht,
                           (((vb >> (2 * c2 + 1)) & 1u) ? 0xFFFF0000u : 0u);
                 pk[c2] = a2;
             }
-            tmem_st4(e.t_a + ch * 4, pk);
+            tmem_st2(e.t_a + ch * 2, pk);
         }
     }
 }

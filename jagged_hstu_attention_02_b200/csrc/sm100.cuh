@@ -249,6 +249,23 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8])
                  : "memory");
 }
 
+// Loads 4 consecutive 32-bit columns of this thread's TMEM lane (wait with tmem_wait_ld).
+__device__ __forceinline__ void tmem_ld4(uint32_t taddr, uint32_t (&r)[4])
+{
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(taddr)
+                 : "memory");
+}
+
+// Stores 2 consecutive 32-bit columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_st2(uint32_t taddr, const uint32_t (&r)[2])
+{
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x2.b32 [%0], {%1, %2};" ::"r"(taddr),
+                 "r"(r[0]), "r"(r[1])
+                 : "memory");
+}
+
 // Stores 4 consecutive 32-bit columns of this thread's TMEM lane.
 __device__ __forceinline__ void tmem_st4(uint32_t taddr, const uint32_t (&r)[4])
 {
@@ -303,6 +320,11 @@ __device__ __forceinline__ void reg_fence(uint32_t (&r)[32])
                    "+r"(r[30]), "+r"(r[31]));
 }
 
+__device__ __forceinline__ void reg_fence(uint32_t (&r)[4])
+{
+    asm volatile("" : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]));
+}
+
 __device__ __forceinline__ void reg_fence(uint32_t (&r)[8])
 {
     asm volatile(""
@@ -345,6 +367,11 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
     uint32_t r;
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
     return r;
+}
+
+__device__ __forceinline__ void st_shared_v2(uint32_t addr, uint32_t a, uint32_t b)
+{
+    asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(addr), "r"(a), "r"(b) : "memory");
 }
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
