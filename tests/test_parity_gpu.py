@@ -298,3 +298,50 @@ def test_fwd_bwd_parity_any_timestamp_order(stamps, dims):
     for got, key in ((dq, "dq"), (dk, "dk"), (dv_, "dv"), (du, "du"), (drel, "drel"),
                      (dtb, "dtb")):
         assert_close(_np(got), ref[key], "bf16", name + " " + key)
+
+
+# ------------------------------------------------------------------ work-unit hand-out
+
+def _fwd_bwd_check(b, name, seqs=None):
+    """Inference and training forward, then backward, against the oracle; with `seqs` the
+    per-token outputs are compared on those sequences only (the table gradients need all)."""
+    dev = ops.batch_to_device(b)
+    out_inf = ops.run_fwd(b, dev)
+    out, saved = ops.run_fwd(b, dev, training=True)
+    g = ops.run_bwd(b, saved, dev_tensors=dev)
+    torch.cuda.synchronize()
+    assert ops.read_device_status(ops.fwd.last_workspace) == 0
+    assert ops.read_device_status(ops.bwd.last_workspace) == 0
+    ref_f = oracle.fwd(b if seqs is None else sub_batch(b, seqs))
+    ref_b = oracle.bwd(b)
+    rows = slice(None) if seqs is None else rows_of(b, seqs)
+    assert_close(_np(out_inf)[rows], ref_f["out"], b.dtype, name + " inference out")
+    assert_close(_np(out)[rows], ref_f["out"], b.dtype, name + " training out")
+    for got, key in zip(g, ["dq", "dk", "dv", "du", "drel", "dtb"]):
+        assert_close(_np(got), ref_b[key], b.dtype, name + " " + key)
+
+
+def test_more_sequences_than_the_tile_cache():
+    """2100 sequences (the per-CTA cache of tile counts holds 2048): every unit is drawn
+    and checked against its sequence; empty sequences and two-tile ones among them."""
+    rng = np.random.default_rng(2100)
+    lengths = rng.integers(0, 41, size=2100)
+    lengths[[5, 700, 2099]] = [129, 200, 150]
+    lengths[[6, 7, 1500]] = 0
+    tgt = np.minimum(rng.integers(0, 4, size=2100), lengths)
+    b = synth.make_batch(rng, lengths, 2, 64, 64, "bf16", contextuals=0, targets=tgt,
+                         rel_bias_len=int(lengths.max()) + 1, time_bias_len=128,
+                         with_dout=True)
+    _fwd_bwd_check(b, "2100 sequences")
+
+
+def test_tile_count_past_the_cache_range():
+    """A sequence of 33,000 tokens has more 128-row tiles than the cache counts (255): its
+    units past that count are checked against the sequence itself.  Windowed, so the
+    oracle stays quick."""
+    rng = np.random.default_rng(33000)
+    lengths = [33000, 17, 300]
+    b = synth.make_batch(rng, lengths, 1, 64, 64, "bf16", contextuals=[2, 0, 1],
+                         targets=[8, 3, 20], max_attn_len=64, rel_bias_len=65,
+                         time_bias_len=128, with_dout=True)
+    _fwd_bwd_check(b, "33000-token sequence")
