@@ -337,6 +337,10 @@ LAUNCHES_PER_STEP = 5
 
 
 def measure_e2e(args, b, ops, torch, kw, flops, world):
+    """Training steps through the public API with every step's inputs copied in from pinned
+    host memory and its results (O, dQ, dK, dV, dU, table gradients) read back.  As a
+    training loop would, the copies run on their own streams into and out of double
+    buffers, so step i's compute overlaps step i+1's inputs and step i-1's results."""
     host = {}
     dt = torch.bfloat16 if b.dtype == "bf16" else torch.float32
     src = dict(q=(b.q, dt), k=(b.k, dt), v=(b.v, dt), u=(b.u, dt), dout=(b.dout, dt),
@@ -349,45 +353,71 @@ def measure_e2e(args, b, ops, torch, kw, flops, world):
             t = t.to(cast)
         host[name] = t.pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in host.values())
-    dev = {n: torch.empty_like(t, device="cuda") for n, t in host.items()}
     T, D = b.u.shape
-    out = torch.empty((T, D), dtype=dt, device="cuda")
-    saved = ops.Saved(torch.empty((T, D), device="cuda"), torch.empty(T, device="cuda"),
-                      torch.empty(T, device="cuda"))
-    grads = (torch.empty(b.q.shape, dtype=dt, device="cuda"),
-             torch.empty(b.k.shape, dtype=dt, device="cuda"),
-             torch.empty(b.v.shape, dtype=dt, device="cuda"),
-             torch.empty(b.u.shape, dtype=dt, device="cuda"),
-             torch.empty(b.rel_bias.shape, device="cuda"),
-             torch.empty(b.time_bias.shape, device="cuda"))
-    results = [out] + list(grads)
-    host_out = [torch.empty(r.shape, dtype=r.dtype, pin_memory=True) for r in results]
+    nbuf = 2
+    dev, outs, saveds, gradss = [], [], [], []
+    for _ in range(nbuf):
+        dev.append({n: torch.empty_like(t, device="cuda") for n, t in host.items()})
+        outs.append(torch.empty((T, D), dtype=dt, device="cuda"))
+        saveds.append(ops.Saved(torch.empty((T, D), device="cuda"),
+                                torch.empty(T, device="cuda"), torch.empty(T, device="cuda")))
+        gradss.append((torch.empty(b.q.shape, dtype=dt, device="cuda"),
+                       torch.empty(b.k.shape, dtype=dt, device="cuda"),
+                       torch.empty(b.v.shape, dtype=dt, device="cuda"),
+                       torch.empty(b.u.shape, dtype=dt, device="cuda"),
+                       torch.empty(b.rel_bias.shape, device="cuda"),
+                       torch.empty(b.time_bias.shape, device="cuda")))
+    results = [[outs[k]] + list(gradss[k]) for k in range(nbuf)]
+    host_out = [torch.empty(r.shape, dtype=r.dtype, pin_memory=True) for r in results[0]]
     d2h = sum(t.numel() * t.element_size() for t in host_out)
+    s_in, s_comp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    in_done = [torch.cuda.Event() for _ in range(nbuf)]
+    comp_done = [torch.cuda.Event() for _ in range(nbuf)]
+    out_done = [torch.cuda.Event() for _ in range(nbuf)]
 
-    def step():
-        for n in host:
-            dev[n].copy_(host[n], non_blocking=True)
-        ops.fwd(dev["q"], dev["k"], dev["v"], dev["u"], dev["seq_offsets"],
-                dev["num_contextuals"], dev["num_targets"], dev["timestamps"], dev["rel_bias"],
-                dev["time_bias"], training=True, out=out, saved=saved, **kw)
-        ops.bwd(dev["dout"], dev["q"], dev["k"], dev["v"], dev["u"], dev["seq_offsets"],
-                dev["num_contextuals"], dev["num_targets"], dev["timestamps"], dev["rel_bias"],
-                dev["time_bias"], saved=saved, grads=grads, **kw)
-        for r, h in zip(results, host_out):
-            h.copy_(r, non_blocking=True)
+    def run(n, start):
+        for st in (s_in, s_comp, s_out):
+            st.wait_event(start)
+        for i in range(n):
+            k = i % nbuf
+            with torch.cuda.stream(s_in):           # step i's inputs, once step i-2 is done
+                if i >= nbuf:
+                    s_in.wait_event(comp_done[k])
+                for name in host:
+                    dev[k][name].copy_(host[name], non_blocking=True)
+                in_done[k].record(s_in)
+            with torch.cuda.stream(s_comp):         # step i, once its results buffer is read
+                s_comp.wait_event(in_done[k])
+                if i >= nbuf:
+                    s_comp.wait_event(out_done[k])
+                d = dev[k]
+                ops.fwd(d["q"], d["k"], d["v"], d["u"], d["seq_offsets"], d["num_contextuals"],
+                        d["num_targets"], d["timestamps"], d["rel_bias"], d["time_bias"],
+                        training=True, out=outs[k], saved=saveds[k], **kw)
+                ops.bwd(d["dout"], d["q"], d["k"], d["v"], d["u"], d["seq_offsets"],
+                        d["num_contextuals"], d["num_targets"], d["timestamps"], d["rel_bias"],
+                        d["time_bias"], saved=saveds[k], grads=gradss[k], **kw)
+                comp_done[k].record(s_comp)
+            with torch.cuda.stream(s_out):          # step i's results back to the host
+                s_out.wait_event(comp_done[k])
+                for r, h in zip(results[k], host_out):
+                    h.copy_(r, non_blocking=True)
+                out_done[k].record(s_out)
 
-    for _ in range(max(args.warmup, 3)):
-        step()
-    torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
-    for _ in range(args.steps):
-        step()
+    run(max(args.warmup, 3), e0)
+    torch.cuda.synchronize()
+    e0.record()
+    run(args.steps, e0)
+    for st in (s_in, s_comp, s_out):
+        torch.cuda.current_stream().wait_stream(st)
     e1.record()
     e1.synchronize()
     ms = e0.elapsed_time(e1) / args.steps
     return {"value": round(world * flops / (ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
-            "ms_per_step": round(ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+            "ms_per_step": round(ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "overlap": "inputs of step i+1 and results of step i-1 copied while step i runs"}
 
 
 def measure_secondary(ops, torch, peaks, rank):
