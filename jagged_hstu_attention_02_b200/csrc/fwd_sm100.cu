@@ -7,15 +7,16 @@
 // time bias and the mask is applied after the nonlinearity, never as -inf before it ("HSTU
 // tensor by tensor: SiLU aggregation, temporal bias and gating", sections "Similar shape,
 // different aggregation" and "Do not copy softmax masking mechanically"); A is rounded to
-// bf16 and written back over S in TMEM (two elements per 32-bit column), and tcgen05 adds
-// A V into an fp32 output accumulator in TMEM with A read from TMEM.  The 1/N scale
+// bf16 and written into its own TMEM columns (two elements per 32-bit column), and tcgen05
+// adds A V into an fp32 output accumulator in TMEM with A read from TMEM.  The 1/N scale
 // ("HSTU-MUSA: HSTU for Moore Threads (MUSA)", "Accuracy Alignment": N = batch max_seqlen)
 // is applied once to the accumulator; Y goes to global memory in fp32.
 //
-// Persistent: one CTA per SM walks the units in longest-first order (query tiles from the
-// last to the first, so the tiles with the most keys start first), so the per-CTA set-up
-// (barriers, TMEM, bias tables, bucket lookup table) happens once per SM and the loads of
-// the next unit (Q is double-buffered) overlap the tail of the current one.  Warp roles (20
+// Persistent: one CTA per SM takes units from a global counter in longest-first order
+// (query tiles from the last to the first, so the tiles with the most keys start first;
+// units.cuh), so the per-CTA set-up (barriers, TMEM, bias tables, bucket lookup table)
+// happens once per SM and the loads of the next unit (Q is double-buffered) overlap the
+// tail of the current one.  Warp roles (20
 // warps): warp 0 lane 0 loads Q and K, warp 2 lane 0 loads V (warp 2 also owns TMEM), warp
 // 1 lane 0 issues the MMAs, warp 3 stages each key tile's timestamps and per-quarter
 // ranges, warps 4-19 are four epilogue warpgroups, each owning 32 of the 128 key columns
