@@ -49,7 +49,9 @@
  * workspace.  fwd/bwd allocate nothing, never synchronise, and only enqueue work on
  * `stream` (a cudaStream_t; NULL = the legacy default stream).  All array pointers are
  * device pointers; `params` is a host pointer read before the call returns.  Device
- * pointers must be 16-byte aligned.
+ * pointers must be 16-byte aligned.  A workspace serves one call at a time: each call resets
+ * the status word and the work-unit counter at its head, so calls that share a workspace
+ * must run in order (one stream, or streams ordered by events).
  *
  * Errors.  Host-checkable problems (NULL required pointer, sizes out of range, misaligned
  * pointer, workspace too small) return a status before anything is enqueued.  Problems in
