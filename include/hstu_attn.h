@@ -55,10 +55,14 @@
  *
  * Errors.  Host-checkable problems (NULL required pointer, sizes out of range, misaligned
  * pointer, workspace too small) return a status before anything is enqueued.  Problems in
- * device-resident data (offsets not monotone or not ending at T, c + t > L, L > max_seqlen)
- * are not fatal: the offending sequence is skipped and a bit is set in the status word at
- * the start of the workspace; hstu_attn_read_device_status() reads it.  No kernel traps,
- * and every wait inside a kernel is bounded.
+ * device-resident data (offsets not monotone, not starting at 0 or not ending at T, c + t > L,
+ * L > max_seqlen) are not fatal: the offending sequence is skipped and a bit is set in the
+ * status word at the start of the workspace; hstu_attn_read_device_status() reads it.  The
+ * rows of a skipped sequence, and rows before seq_offsets[0] or from seq_offsets[B] on, get
+ * zeros in out, saved_y, dk and dv (and the matching mean 0, rstd 1/sqrt(eps), dq 0, du 0),
+ * so every output row is defined while the offsets are non-decreasing; where sequences
+ * overlap, their rows are unspecified.  No kernel traps, and every wait inside a kernel is
+ * bounded.
  */
 #ifndef HSTU_ATTN_H
 #define HSTU_ATTN_H
@@ -154,6 +158,26 @@ hstu_status_t hstu_attn_debug_mask(const hstu_attn_params_t *params, const int64
                                    int32_t seq, int32_t seq_len, uint32_t *bits, void *stream);
 
 /*
+ * Test hook: the mask of sequence `seq` as the tensor-core kernels decide it (bf16 inputs,
+ * d_qk and d_v in {64, 128}): a pair is valid when the kernel visits its 128 x 128 tile and
+ * the 32-wide block the pair lies in marks it.  kernel = 0 selects the forward's decisions
+ * (per query row and 32-key block), kernel = 1 the backward's (per key and 32-query block).
+ * Writes rows [row_begin, row_begin + row_count) x keys [0, key_count) of the mask, row-major,
+ * bit j of row r at word r * key_count / 32 + j / 32, bit j % 32, into `bits` (device,
+ * row_count * key_count / 32 words).  Rows and keys past the sequence's end are included (up
+ * to the tile padding, 128 * ceil(L / 128)): a kernel must never mark them valid for a row
+ * (forward) or key (backward) it stores.  key_count must be a multiple of 32; row_begin and
+ * row_count are >= 0.  Enqueued on `stream`; the same mask as "HSTU-MUSA: HSTU for Moore
+ * Threads (MUSA)", section "Mathematical Equivalence", when the kernels are correct.
+ */
+hstu_status_t hstu_attn_debug_kernel_mask(const hstu_attn_params_t *params,
+                                          const int64_t *seq_offsets,
+                                          const int32_t *num_contextuals,
+                                          const int32_t *num_targets, int32_t seq,
+                                          int32_t kernel, int32_t row_begin, int32_t row_count,
+                                          int32_t key_count, uint32_t *bits, void *stream);
+
+/*
  * Host helper: the time-bucket thresholds the device compares against.  out[k-1] is the
  * smallest |dt| whose bucket is >= k, for k = 1..nb-1, with the bucket decided in fp64
  * exactly as floor(log((double)|dt| + 1.0) / div) (UINT64_MAX when never reached).
@@ -173,7 +197,8 @@ hstu_status_t hstu_attn_time_thresholds(double div, int32_t nb, uint64_t *out);
  *   - Limit: the scratch need is 256 + 4 * total_tokens * num_heads * d_v bytes; a request
  *     above 32 MiB returns HSTU_ERR_WORKSPACE_TOO_SMALL before anything is enqueued.
  *   - Set-up: the first call on each device looks up the array's device address (with that
- *     device current); make that first call before any stream capture.
+ *     device current), and so does the first call after that device's context was reset
+ *     (cudaDeviceReset); make those calls before any stream capture.
  *   - Sharing: all calls on a device share the one array, which keeps the last call's
  *     contents (the status word is cleared by every call).  Calls that overlap on the GPU
  *     (other streams, other threads) race on it: serialise them.
@@ -202,6 +227,18 @@ hstu_status_t hstu_attn_fwd_noalloc(const hstu_attn_params_t *params, const void
  * graph nodes of their own, so every replay of the graph stamps them.
  */
 hstu_status_t hstu_attn_set_stage_events(int32_t stage, void *start_event, void *stop_event);
+
+/*
+ * Test hook for the bounded waits.  limit_cycles (> 0) replaces, for every later fwd/bwd
+ * launch, the number of SM clock cycles a pipeline wait inside the tensor-core kernels may
+ * take before the kernel gives up (0 restores the default, about 2 s); the waits that let
+ * copies and MMAs in flight finish before a block exits keep the default.  stall = 1 makes
+ * the MMA issuer of those kernels first wait on a barrier that nothing completes, so that
+ * wait runs out, HSTU_DEV_WAIT_TIMEOUT is set in the status word and every role of the
+ * kernel unwinds as after any timeout (outputs then unspecified); stall = 0 turns it off.
+ * Process-wide and not thread-safe: for tests only.
+ */
+hstu_status_t hstu_attn_set_wait_test(int64_t limit_cycles, int32_t stall);
 
 /* Static description of a status code. */
 const char *hstu_status_string(hstu_status_t status);

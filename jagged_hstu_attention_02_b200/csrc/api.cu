@@ -10,6 +10,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "sm100.cuh"
 
 namespace hstu {
 
@@ -82,6 +83,10 @@ hstu_status_t validate(const hstu_attn_params_t *p)
     return HSTU_OK;
 }
 
+// Test hook state (hstu_attn_set_wait_test): the pipeline-wait limit and the stall switch.
+long long g_wait_limit = sm100::kWaitLimitCycles;
+int32_t g_stall_test = 0;
+
 DevParams make_dev_params(const hstu_attn_params_t *p, const int64_t *offsets, const int32_t *ctx,
                           const int32_t *tgt, const int64_t *ts, const float *rel,
                           const float *tb, void *workspace)
@@ -108,6 +113,8 @@ DevParams make_dev_params(const hstu_attn_params_t *p, const int64_t *offsets, c
     d.rel = rel;
     d.tb = tb;
     d.status = reinterpret_cast<int32_t *>(workspace);
+    d.wait_limit = g_wait_limit;
+    d.stall_test = g_stall_test;
     if (d.NB > 0) {
         const ThrEntry &e = thresholds(p->time_bucket_div, d.NB);
         d.n_thr = e.n_reach;
@@ -195,6 +202,14 @@ hstu_status_t hstu_attn_time_thresholds(double div, int32_t nb, uint64_t *out)
         return HSTU_ERR_INVALID_ARGUMENT;
     const ThrEntry &e = thresholds(div, nb);
     for (int k = 0; k < nb - 1; ++k) out[k] = e.thr[k];
+    return HSTU_OK;
+}
+
+hstu_status_t hstu_attn_set_wait_test(int64_t limit_cycles, int32_t stall)
+{
+    if (limit_cycles < 0 || (stall != 0 && stall != 1)) return HSTU_ERR_INVALID_ARGUMENT;
+    g_wait_limit = limit_cycles == 0 ? sm100::kWaitLimitCycles : (long long)limit_cycles;
+    g_stall_test = stall;
     return HSTU_OK;
 }
 
@@ -383,6 +398,26 @@ hstu_status_t hstu_attn_debug_mask(const hstu_attn_params_t *p, const int64_t *s
     DevParams d = make_dev_params(p, seq_offsets, num_contextuals, num_targets, nullptr, nullptr,
                                   nullptr, nullptr);
     HSTU_CUDA_TRY(launch_debug_mask(d, seq, seq_len, bits, reinterpret_cast<cudaStream_t>(stream)));
+    return HSTU_OK;
+}
+
+hstu_status_t hstu_attn_debug_kernel_mask(const hstu_attn_params_t *p,
+                                          const int64_t *seq_offsets,
+                                          const int32_t *num_contextuals,
+                                          const int32_t *num_targets, int32_t seq,
+                                          int32_t kernel, int32_t row_begin, int32_t row_count,
+                                          int32_t key_count, uint32_t *bits, void *stream)
+{
+    hstu_status_t st = validate(p);
+    if (st != HSTU_OK) return st;
+    if (!seq_offsets || !bits || seq < 0 || seq >= p->batch || (kernel != 0 && kernel != 1) ||
+        row_begin < 0 || row_count < 0 || key_count < 0 || key_count % 32 != 0)
+        return HSTU_ERR_INVALID_ARGUMENT;
+    if (row_count == 0 || key_count == 0) return HSTU_OK;
+    DevParams d = make_dev_params(p, seq_offsets, num_contextuals, num_targets, nullptr, nullptr,
+                                  nullptr, nullptr);
+    HSTU_CUDA_TRY(launch_debug_kernel_mask(d, seq, kernel, row_begin, row_count, key_count, bits,
+                                           reinterpret_cast<cudaStream_t>(stream)));
     return HSTU_OK;
 }
 

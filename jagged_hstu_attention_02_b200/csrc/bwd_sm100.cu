@@ -35,9 +35,9 @@
 
 #include <cstring>
 
-#include "bias.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
+#include "tiles.cuh"
 #include "units.cuh"
 
 namespace hstu {
@@ -48,6 +48,7 @@ namespace {
 
 constexpr int BM = 128, BN = 128;
 constexpr int QW = 32;                  // query columns per epilogue warpgroup
+static_assert(BM == kTile && BN == kTile && QW == kBlk, "tile shapes of tiles.cuh");
 constexpr int kEpiWarps = 16;
 constexpr int kEpiWarp0 = 3;            // warps 0-2: TMA, MMA, TMEM owner + query stamps
 constexpr int kThreads = 32 * (kEpiWarp0 + kEpiWarps);
@@ -63,7 +64,8 @@ enum Bar {
     EPI_DONE = 7,                                                                     // +2
     P_FULL = 9, DQ_FULL = 10, DQ_FREE = 11, ACC_FULL = 12, ACC_FREE = 13, MMA_DONE = 14,
     UNIT_FULL = 15, UNIT_EMPTY = 19,                                                  // +4
-    NUM_BARS = 23
+    NEVER = 23,   // nothing arrives on it (the stall test's wait)
+    NUM_BARS = 24
 };
 
 // Time-stamp ranges of the four 32-query quarters of a query tile.
@@ -111,20 +113,6 @@ struct BwdTcArgs {
     float *tb_slots;               // [gridDim.x, kMaxTimeBuckets] scratch, one row per CTA
     unsigned long long *unit_ctr;  // next work unit to hand out (zeroed by the caller)
     int nkt;                       // key tiles of the longest admissible sequence
-};
-
-// The query tiles [i0, i0+BM) that see key tile [j0, j0+BN), in order.
-struct QTileIter {
-    const SeqInfo &s;
-    int j0, W, qt, nqt;
-    __device__ QTileIter(const SeqInfo &s_, int j0_, int W_)
-        : s(s_), j0(j0_), W(W_), qt(-1), nqt((s_.L + BM - 1) / BM) {}
-    __device__ bool next()
-    {
-        while (++qt < nqt)
-            if (tile_any_valid(qt * BM, qt * BM + BM - 1, j0, j0 + BN - 1, s, W)) return true;
-        return false;
-    }
 };
 
 __device__ __forceinline__ void report_timeout(const DevParams &p)
@@ -478,6 +466,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     }
     fill_seq_tiles(p, kThreads);
+    for (int b = blockIdx.x; b < p.B; b += gridDim.x) {   // rows no unit writes: zero dK, dV
+        RowRange rr[3];
+        const int n = skipped_rows(p, b, rr);
+        for (int x = 0; x < n; ++x) {
+            zero_rows(args.dk, (int64_t)p.H * p.dqk, rr[x], threadIdx.x, kThreads);
+            zero_rows(args.dv, (int64_t)p.H * p.dv, rr[x], threadIdx.x, kThreads);
+        }
+    }
     __threadfence();   // the zeroed slot row is in place before any reduction into it
     __syncthreads();
     if (p.NB > 0) build_lut(thr, p.n_thr, lut, lut_valid);
@@ -504,7 +500,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = true;
             while (ok && un.next()) {
                 const int row0 = (int)un.s.start, j0 = un.tile * BN;
-                if (n >= 1 && !mbar_wait(&bars[KV_EMPTY], (n - 1) & 1)) { ok = false; break; }
+                if (n >= 1 && !mbar_wait(&bars[KV_EMPTY], (n - 1) & 1, p.wait_limit)) { ok = false; break; }
                 mbar_arrive_expect_tx(&bars[KV_FULL], L::KB + L::VB);
                 for (int kb = 0; kb < DQK / 64; ++kb)
                     tma_load_3d(sm + L::K_OFF + kb * kBlockBytes, &args.tk, &bars[KV_FULL],
@@ -515,7 +511,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ++n;
                 QTileIter t(un.s, j0, p.W);
                 while (t.next()) {
-                    if (g >= 1 && !mbar_wait(&bars[QD_EMPTY], (g - 1) & 1)) { ok = false; break; }
+                    if (g >= 1 && !mbar_wait(&bars[QD_EMPTY], (g - 1) & 1, p.wait_limit)) { ok = false; break; }
                     const int i0 = t.qt * BM;
                     mbar_arrive_expect_tx(&bars[QD_FULL], L::QB + 2 * L::YB);
                     for (int kb = 0; kb < DQK / 64; ++kb)
@@ -533,8 +529,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!ok || !un.ok) report_timeout(p);
             // every copy has landed before the CTA may exit
             bool drained = true;
-            if (n >= 1) drained &= mbar_wait(&bars[KV_FULL], (n - 1) & 1);
-            if (g >= 1) drained &= mbar_wait(&bars[QD_FULL], (g - 1) & 1);
+            if (n >= 1) drained &= mbar_wait(&bars[KV_FULL], (n - 1) & 1, kWaitLimitCycles);
+            if (g >= 1) drained &= mbar_wait(&bars[QD_FULL], (g - 1) & 1, kWaitLimitCycles);
             if (!drained) report_timeout(p);
         }
     } else if (warp == 1) {
@@ -549,16 +545,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t yl_addr = sm_base + L::YL_OFF, ds_addr = sm_base + L::YL_OFF;
             UnitFeed<FEED_THREAD, true, BN> un(p, ring, args.nkt);
             int n = 0, g = 0;
-            bool ok = true;
+            // the stall test: a wait that runs out, then the same unwinding as any timeout
+            bool ok = !p.stall_test || mbar_wait(&bars[NEVER], 0, p.wait_limit);
             while (ok && un.next()) {
-                if (!mbar_wait(&bars[KV_FULL], n & 1)) { ok = false; break; }
+                if (!mbar_wait(&bars[KV_FULL], n & 1, p.wait_limit)) { ok = false; break; }
                 QTileIter t(un.s, un.tile * BN, p.W);
                 int x = 0;
                 while (t.next()) {
-                    if (!mbar_wait(&bars[QD_FULL], g & 1)) { ok = false; break; }
+                    if (!mbar_wait(&bars[QD_FULL], g & 1, p.wait_limit)) { ok = false; break; }
                     // the previous tile's dQ has been read: every MMA of it completed, so the
                     // S^T/A^T and dP^T/dQ columns are free
-                    if (g >= 1 && !mbar_wait(&bars[DQ_FREE], (g - 1) & 1)) { ok = false; break; }
+                    if (g >= 1 && !mbar_wait(&bars[DQ_FREE], (g - 1) & 1, p.wait_limit)) { ok = false; break; }
                     tc_fence_after();
 #pragma unroll
                     for (int kb = 0; kb < DQK / 64; ++kb)
@@ -580,9 +577,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                             umma_bf16_ss(tmem + kColDP, a, bl, id_s, 1u);
                         }
                     umma_commit(&bars[SD_FULL]);
-                    if (!mbar_wait(&bars[P_FULL], g & 1)) { ok = false; break; }
+                    if (!mbar_wait(&bars[P_FULL], g & 1, p.wait_limit)) { ok = false; break; }
                     // dV and dK of the previous unit have been read out
-                    if (x == 0 && n >= 1 && !mbar_wait(&bars[ACC_FREE], (n - 1) & 1)) {
+                    if (x == 0 && n >= 1 && !mbar_wait(&bars[ACC_FREE], (n - 1) & 1, p.wait_limit)) {
                         ok = false;
                         break;
                     }
@@ -621,7 +618,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (!ok || !un.ok) report_timeout(p);
             umma_commit(&bars[MMA_DONE]);
-            if (!mbar_wait(&bars[MMA_DONE], 0)) report_timeout(p);
+            if (!mbar_wait(&bars[MMA_DONE], 0, kWaitLimitCycles)) report_timeout(p);
         }
     } else if (warp == 2) {
         // -------------------------------------------------------------------- query stamps
@@ -635,7 +632,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             while (t.next()) {
                 const int st = g & 1;
                 // the epilogue has finished with the stamps of tile g - 2
-                if (g >= 2 && !warp_wait(&bars[EPI_DONE + st], ((g >> 1) - 1) & 1)) {
+                if (g >= 2 && !warp_wait(&bars[EPI_DONE + st], ((g >> 1) - 1) & 1, p.wait_limit)) {
                     ok = false;
                     break;
                 }
@@ -707,8 +704,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             int x = 0;
             while (t.next()) {
                 const int st = g & 1;
-                if (!warp_wait(&bars[META_FULL + st], (g >> 1) & 1) ||
-                    !warp_wait(&bars[SD_FULL], g & 1)) {
+                if (!warp_wait(&bars[META_FULL + st], (g >> 1) & 1, p.wait_limit) ||
+                    !warp_wait(&bars[SD_FULL], g & 1, p.wait_limit)) {
                     ok = false;
                     break;
                 }
@@ -720,8 +717,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     e.t_dp = tl + kColDP + wq * QW;
                     e.ds_row = sm_base + L::YL_OFF + (wq >> 1) * kBlockBytes + r * 128;
                     e.ds_chunk0 = (wq & 1) * 4;
-                    e.full = tile_all_valid(e.iq, e.iq + QW - 1, j0, j0 + BN - 1, s, p.W);
-                    e.vbits = e.full ? 0xFFFFFFFFu : (uint32_t)col_valid_bits(k.j, e.iq, s, p.W);
+                    const BlockMask bm = bwd_block_mask(s, j0, e.iq, k.j, p.W);
+                    e.full = bm.full;
+                    e.vbits = bm.bits;
                     const uint32_t vb = e.vbits;
                     const bool idle = vb == 0u;
                     if (!__any_sync(0xffffffffu, !idle)) {
@@ -796,7 +794,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 warp_arrive(&bars[EPI_DONE + st]);
 
                 // ---- dQ tile: lanes = query rows of this tile; columns split by warpgroup
-                if (!warp_wait(&bars[DQ_FULL], g & 1)) { ok = false; break; }
+                if (!warp_wait(&bars[DQ_FULL], g & 1, p.wait_limit)) { ok = false; break; }
                 tc_fence_after();
                 {
                     constexpr int QC = DQK / kGroups;          // 16, 32 or 64 columns
@@ -834,7 +832,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!ok) break;
             if (use_ts && k.run != 0.f) red_add(tb_slot + k.cur_b, k.run);
             // ---- dV and dK of the key rows (every key tile sees at least its diagonal tile)
-            if (!warp_wait(&bars[ACC_FULL], n & 1)) { ok = false; break; }
+            if (!warp_wait(&bars[ACC_FULL], n & 1, p.wait_limit)) { ok = false; break; }
             tc_fence_after();
             {
                 constexpr int VC = DV / kGroups, KC = DQK / kGroups;

@@ -31,6 +31,8 @@ struct DevParams {
     const int64_t *ts;
     const float *rel, *tb;
     int32_t *status;
+    long long wait_limit;   // cycles a pipeline wait may take before the kernel gives up
+    int32_t stall_test;     // test only: the MMA issuer first waits on a barrier nothing completes
     // smallest |dt| of bucket k+1 (fp64-decided on the host), ascending
     uint64_t thr[kMaxTimeBuckets - 1];
 };
@@ -58,6 +60,8 @@ __device__ __forceinline__ SeqInfo load_seq(const DevParams &p, int b, bool repo
     s.ok = true;
     int bits = 0;
     if (a < 0 || L < 0 || e > p.T) { bits |= HSTU_DEV_BAD_OFFSETS; }
+    // the offsets must start at row 0 and end at row T
+    if ((b == 0 && a != 0) || (b == p.B - 1 && e != p.T)) { bits |= HSTU_DEV_BAD_OFFSETS; }
     if (L > p.N) { bits |= HSTU_DEV_SEQ_TOO_LONG; }
     if (bits == 0 && (s.c < 0 || s.t < 0 || (int64_t)s.c + s.t > L)) bits |= HSTU_DEV_BAD_COUNTS;
     if (bits) {
@@ -68,6 +72,35 @@ __device__ __forceinline__ SeqInfo load_seq(const DevParams &p, int b, bool repo
     s.L = (int)L;
     s.E = s.L - s.t;
     return s;
+}
+
+// Token rows that sequence b leaves without a computed output, clipped to [0, T): its own
+// rows when it is skipped for invalid data, and for the first (last) sequence the rows
+// before seq_offsets[0] (from seq_offsets[B] on).  The kernels that write per-token outputs
+// zero these rows, so that every output row is defined whenever the offsets are
+// non-decreasing (overlapping sequences leave the overlap unspecified).
+struct RowRange {
+    int64_t a, e;
+};
+
+__device__ __forceinline__ int skipped_rows(const DevParams &p, int b, RowRange (&r)[3])
+{
+    int n = 0;
+    const int64_t a = p.offsets[b], e = p.offsets[b + 1];
+    if (!load_seq(p, b, false).ok) r[n++] = RowRange{max(a, (int64_t)0), min(e, p.T)};
+    if (b == 0 && a > 0) r[n++] = RowRange{0, min(a, p.T)};
+    if (b == p.B - 1 && e < p.T) r[n++] = RowRange{max(e, (int64_t)0), p.T};
+    return n;
+}
+
+// Zeroes rows [r.a, r.e) of a row-major array with `width` elements per row, element-wise
+// by `nthr` threads (tid = this thread's index among them).  Rare path: invalid data only.
+template <typename T>
+__device__ __forceinline__ void zero_rows(T *base, int64_t width, const RowRange &r, int tid,
+                                          int nthr)
+{
+    if (!base || r.e <= r.a) return;
+    for (int64_t x = r.a * width + tid; x < r.e * width; x += nthr) base[x] = T(0.f);
 }
 
 // Tiles of 128 rows of each sequence (ceil(L/128), saturated at 255; 0 for an invalid

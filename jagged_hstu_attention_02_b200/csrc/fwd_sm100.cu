@@ -32,11 +32,12 @@
 // timeout sets HSTU_DEV_WAIT_TIMEOUT and the CTA unwinds.
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cstring>
 
-#include "bias.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
+#include "tiles.cuh"
 #include "units.cuh"
 
 namespace hstu {
@@ -46,6 +47,7 @@ using namespace sm100;
 namespace {
 
 constexpr int BM = 128, BN = 128, QW = 32;   // QW: key columns per epilogue warpgroup
+static_assert(BM == kTile && BN == kTile && QW == kBlk, "tile shapes of tiles.cuh");
 constexpr int kEpiWarps = 16;                  // four warpgroups
 constexpr int kTcThreads = 128 + 32 * kEpiWarps;
 constexpr int kRelSmemMax = 4352;   // covers N up to 4351 (R = N + 1)
@@ -60,7 +62,9 @@ constexpr float kTruncBump = 1.0028f;
 enum Bar { Q_FULL = 0, Q_EMPTY = 2, K_FULL = 4, K_EMPTY = 6, V_FULL = 8, V_EMPTY = 10,
            S_FULL = 12, S_FREE = 14, P_FULL = 16, P_FREE = 18, META_FULL = 20, EPI_DONE = 22,
            O_FULL = 24, O_FREE = 25, MMA_DONE = 26, UNIT_FULL = 27, UNIT_EMPTY = 31,  // +4
-           NUM_BARS = 35 };
+           NEVER = 35,   // nothing arrives on it (the stall test's wait)
+           NUM_BARS = 36 };
+static_assert(NUM_BARS <= 40, "barrier area");
 
 struct TileMeta {
     int64_t tmin[4], tmax[4];   // timestamp range of each 32-key quarter (valid keys only)
@@ -95,27 +99,6 @@ struct FwdTcArgs {
     float *y;
     unsigned long long *unit_ctr;   // next work unit to hand out (zeroed by the caller)
     int nqt;   // query tiles of the longest admissible sequence: ceil(N / 128)
-};
-
-// Visits the key tiles of query tile [i0, i0+BM) that hold a valid pair, in order.
-struct TileIter {
-    const SeqInfo &s;
-    int i0, W, kt;
-    // Valid pairs have j <= i, except contextual rows, which see the whole contextual
-    // prefix: the first candidate key tile is the later of the diagonal and the prefix's end.
-    __device__ TileIter(const SeqInfo &s_, int i0_, int W_)
-        : s(s_), i0(i0_), W(W_),
-          kt(min((s_.L + BN - 1) / BN, max(i0_ / BN, (s_.c - 1) / BN) + 1)) {}
-    // Descending: the diagonal tile, the most expensive one of a unit (masks, clamped
-    // positions, many time buckets), comes first, where the double-buffered S and A absorb
-    // the spread between warps, instead of last, where every warp would wait for the
-    // slowest one before the unit's output can be read.
-    __device__ bool next()
-    {
-        while (--kt >= 0)
-            if (tile_any_valid(i0, i0 + BM - 1, kt * BN, kt * BN + BN - 1, s, W)) return true;
-        return false;
-    }
 };
 
 __device__ __forceinline__ void report_timeout(const DevParams &p)
@@ -287,6 +270,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (int x = threadIdx.x; x < p.R; x += kTcThreads) relh[x] = tscale * p.rel[x];
     if (p.R == 0 && threadIdx.x == 0) relh[0] = 0.f;   // read, times zero bias, without a table
     fill_seq_tiles(p, kTcThreads);
+    for (int b = blockIdx.x; b < p.B; b += gridDim.x) {   // rows no unit writes: zero Y
+        RowRange rr[3];
+        const int n = skipped_rows(p, b, rr);
+        for (int x = 0; x < n; ++x) zero_rows(args.y, p.D, rr[x], threadIdx.x, kTcThreads);
+    }
     __syncthreads();
     if (p.NB > 0) build_lut(thr, p.n_thr, lutp, lut_valid);
     grid_dep_release();   // the LayerNorm behind this kernel may be scheduled
@@ -306,7 +294,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             bool ok = true;
             while (ok && un.next()) {
                 const int i0 = un.tile * BM, row0 = (int)un.s.start, qs = n % QST;
-                if (n >= QST && !mbar_wait(&bars[Q_EMPTY + qs], (n / QST - 1) & 1)) {
+                if (n >= QST && !mbar_wait(&bars[Q_EMPTY + qs], (n / QST - 1) & 1, p.wait_limit)) {
                     ok = false;
                     break;
                 }
@@ -317,7 +305,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 TileIter t(un.s, i0, p.W);
                 while (t.next()) {
                     const int st = g % KST;
-                    if (g >= KST && !mbar_wait(&bars[K_EMPTY + st], (g / KST - 1) & 1)) {
+                    if (g >= KST && !mbar_wait(&bars[K_EMPTY + st], (g / KST - 1) & 1, p.wait_limit)) {
                         ok = false;
                         break;
                     }
@@ -333,9 +321,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             // loads issued must land before the CTA exits (bounded)
             bool drained = true;
             for (int x = n - 1; x >= 0 && x >= n - QST; --x)
-                drained &= mbar_wait(&bars[Q_FULL + x % QST], (x / QST) & 1);
+                drained &= mbar_wait(&bars[Q_FULL + x % QST], (x / QST) & 1, kWaitLimitCycles);
             for (int x = g - 1; x >= 0 && x >= g - KST; --x)
-                drained &= mbar_wait(&bars[K_FULL + x % KST], (x / KST) & 1);
+                drained &= mbar_wait(&bars[K_FULL + x % KST], (x / KST) & 1, kWaitLimitCycles);
             if (!drained) report_timeout(p);
         }
     } else if (warp == 2) {
@@ -350,7 +338,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 TileIter t(un.s, un.tile * BM, p.W);
                 while (t.next()) {
                     const int st = g % VST;
-                    if (g >= VST && !mbar_wait(&bars[V_EMPTY + st], (g / VST - 1) & 1)) {
+                    if (g >= VST && !mbar_wait(&bars[V_EMPTY + st], (g / VST - 1) & 1, p.wait_limit)) {
                         ok = false;
                         break;
                     }
@@ -364,7 +352,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             if (!ok || !un.ok) report_timeout(p);
             bool drained = true;
             for (int x = g - 1; x >= 0 && x >= g - VST; --x)
-                drained &= mbar_wait(&bars[V_FULL + x % VST], (x / VST) & 1);
+                drained &= mbar_wait(&bars[V_FULL + x % VST], (x / VST) & 1, kWaitLimitCycles);
             if (!drained) report_timeout(p);
         }
     }
@@ -377,9 +365,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             // A V for tile g of unit n; first/last tile of the unit
             auto issue_pv = [&](int g, int n, bool first, bool last) -> bool {
                 const int ps = g % NP;
-                if (!mbar_wait(&bars[P_FULL + ps], (g / NP) & 1)) return false;
-                if (!mbar_wait(&bars[V_FULL + g % VST], (g / VST) & 1)) return false;
-                if (first && n >= 1 && !mbar_wait(&bars[O_FREE], (n - 1) & 1)) return false;
+                if (!mbar_wait(&bars[P_FULL + ps], (g / NP) & 1, p.wait_limit)) return false;
+                if (!mbar_wait(&bars[V_FULL + g % VST], (g / VST) & 1, p.wait_limit)) return false;
+                if (first && n >= 1 && !mbar_wait(&bars[O_FREE], (n - 1) & 1, p.wait_limit)) return false;
                 tc_fence_after();
                 const uint32_t v_addr = sm_base + L::V_OFF + (g % VST) * L::VB;
 #pragma unroll
@@ -399,21 +387,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             };
             UnitFeed<FEED_THREAD, false, BM> un(p, ring, args.nqt);
             int n = 0, g = 0;
-            bool ok = true;
+            // the stall test: a wait that runs out, then the same unwinding as any timeout
+            bool ok = !p.stall_test || mbar_wait(&bars[NEVER], 0, p.wait_limit);
             bool pend = false;                  // an A V waiting for its A
             int pg = 0, pn = 0;
             bool pfirst = false;
             while (ok && un.next()) {
                 const int qs = n % QST;
-                if (!mbar_wait(&bars[Q_FULL + qs], (n / QST) & 1)) { ok = false; break; }
+                if (!mbar_wait(&bars[Q_FULL + qs], (n / QST) & 1, p.wait_limit)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t q_addr = sm_base + L::Q_OFF + qs * L::QB;
                 TileIter t(un.s, un.tile * BM, p.W);
                 bool first = true, more = t.next();
                 while (more) {
                     const int st = g & 1, ks = g % KST;
-                    if (!mbar_wait(&bars[K_FULL + ks], (g / KST) & 1) ||
-                        (g >= 2 && !mbar_wait(&bars[S_FREE + st], ((g >> 1) - 1) & 1))) {
+                    if (!mbar_wait(&bars[K_FULL + ks], (g / KST) & 1, p.wait_limit) ||
+                        (g >= 2 && !mbar_wait(&bars[S_FREE + st], ((g >> 1) - 1) & 1, p.wait_limit))) {
                         ok = false;
                         break;
                     }
@@ -446,7 +435,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             if (!ok || !un.ok) report_timeout(p);
             // every MMA issued must complete before TMEM is released (bounded)
             umma_commit(&bars[MMA_DONE]);
-            if (!mbar_wait(&bars[MMA_DONE], 0)) report_timeout(p);
+            if (!mbar_wait(&bars[MMA_DONE], 0, kWaitLimitCycles)) report_timeout(p);
         }
     } else if (warp == 3) {
         // -------------------------------------------------------------------- tile metadata
@@ -460,7 +449,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             while (t.next()) {
                 const int st = g & 1;
                 // the epilogue is done with this stage's stamps (tile g - 2)
-                if (g >= 2 && !warp_wait(&bars[EPI_DONE + st], ((g >> 1) - 1) & 1)) {
+                if (g >= 2 && !warp_wait(&bars[EPI_DONE + st], ((g >> 1) - 1) & 1, p.wait_limit)) {
                     report_timeout(p);
                     ok = false;
                     break;
@@ -534,14 +523,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             while (t.next()) {
                 const int st = g & 1, ps = g % NP;
                 const int jq = t.kt * BN + wq * QW;      // first key of this warpgroup's quarter
-                const bool full = tile_all_valid(i0, i0 + BM - 1, jq, jq + QW - 1, s, p.W);
+                const BlockMask bm = fwd_block_mask(s, i0, jq, i, p.W);
+                const bool full = bm.full;
                 // the set-up below needs only the stamps; S is waited for afterwards
-                if (!warp_wait(&bars[META_FULL + st], (g >> 1) & 1)) {
+                if (!warp_wait(&bars[META_FULL + st], (g >> 1) & 1, p.wait_limit)) {
                     ok = false;
                     break;
                 }
                 // ---- per (row, quarter tile) structure; path choices are made warp-uniform
-                const uint32_t vmask = full ? 0xFFFFFFFFu : (uint32_t)row_valid_bits(i, jq, s, p.W);
+                const uint32_t vmask = bm.bits;
                 const int rbase = pi - jq;            // rel index of key jq + c is rbase - c
                 // a 32 x 32 block without a valid pair only writes zeros into A
                 const bool blk_any = __any_sync(0xffffffffu, vmask != 0u);
@@ -573,8 +563,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 e.n_thr = p.n_thr;
                 e.tsi = tsi;
                 // S of this tile; A's buffer is free once the A V of tile g - NP has completed
-                if (!warp_wait(&bars[S_FULL + st], (g >> 1) & 1) ||
-                    (g >= NP && !warp_wait(&bars[P_FREE + ps], ((g / NP) - 1) & 1))) {
+                if (!warp_wait(&bars[S_FULL + st], (g >> 1) & 1, p.wait_limit) ||
+                    (g >= NP && !warp_wait(&bars[P_FREE + ps], ((g / NP) - 1) & 1, p.wait_limit))) {
                     ok = false;
                     break;
                 }
@@ -608,7 +598,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             }
             if (!ok) break;
             // ---- the unit's output: Y = (1/N) O; this warpgroup's quarter of the columns
-            if (!warp_wait(&bars[O_FULL], n & 1)) { ok = false; break; }
+            if (!warp_wait(&bars[O_FULL], n & 1, p.wait_limit)) { ok = false; break; }
             tc_fence_after();
             constexpr int OC = DV / 4;                // 32 or 16 output columns per warpgroup
             uint32_t ro[32];
@@ -658,16 +648,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
 int num_sms()
 {
-    static int n = 0;
-    if (n == 0) {
-        int dev = 0, v = 0;
-        if (cudaGetDevice(&dev) == cudaSuccess &&
-            cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0)
-            n = v;
-        else
-            return 148;
+    // cached per device ordinal (a process may drive GPUs of different sizes)
+    constexpr int kMaxDev = 64;
+    static std::atomic<int> cache[kMaxDev];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 148;
+    if (dev < kMaxDev) {
+        const int v = cache[dev].load(std::memory_order_relaxed);
+        if (v > 0) return v;
     }
-    return n;
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+        return 148;
+    if (dev < kMaxDev) cache[dev].store(v, std::memory_order_relaxed);
+    return v;
 }
 
 namespace {

@@ -114,5 +114,9 @@ bool encode_tmap_bf16(CUtensorMap *m, const void *base, int d, int H, int64_t T)
 
 cudaError_t launch_debug_mask(const DevParams &p, int seq, int seq_len, uint32_t *bits,
                               cudaStream_t st);
+// Mask of rows [row0, row0 + nrows) x keys [0, nkeys) (nkeys a multiple of 32) of sequence
+// seq as the tensor-core forward (kernel 0) or backward (kernel 1) decides it.
+cudaError_t launch_debug_kernel_mask(const DevParams &p, int seq, int kernel, int row0,
+                                     int nrows, int nkeys, uint32_t *bits, cudaStream_t st);
 
 }  // namespace hstu

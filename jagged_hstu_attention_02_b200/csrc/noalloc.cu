@@ -8,6 +8,8 @@
 // same forward with its scratch taken from a fixed array in device memory that the library
 // itself declares at file scope.  Every GPU that loads this library keeps that array for
 // the lifetime of the process.
+#include <cudaTypedefs.h>
+
 #include <mutex>
 
 #include "common.cuh"
@@ -23,22 +25,49 @@ constexpr int kMaxDevices = 64;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 std::mutex g_noalloc_mu;
-void *g_noalloc_ptr[kMaxDevices];   // device address of the array, per device
+void *g_noalloc_ptr[kMaxDevices];                 // device address of the array, per device
+unsigned long long g_noalloc_ctx[kMaxDevices];    // id of the context it was looked up in
+
+// Unique id of the calling thread's current context (0 when it cannot be told).  A device
+// reset destroys the context and, with it, the array's address; a new context gets a new
+// id, so the address is looked up again.
+unsigned long long current_context_id()
+{
+    static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+    static PFN_cuCtxGetId_v12000 get_id = nullptr;
+    if (!get_current || !get_id) {
+        void *a = nullptr, *b = nullptr;
+        cudaDriverEntryPointQueryResult qa, qb;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &a, cudaEnableDefault, &qa) != cudaSuccess ||
+            qa != cudaDriverEntryPointSuccess ||
+            cudaGetDriverEntryPoint("cuCtxGetId", &b, cudaEnableDefault, &qb) != cudaSuccess ||
+            qb != cudaDriverEntryPointSuccess)
+            return 0;
+        get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(a);
+        get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(b);
+    }
+    CUcontext c = nullptr;
+    unsigned long long id = 0;
+    if (get_current(&c) != CUDA_SUCCESS || !c || get_id(c, &id) != CUDA_SUCCESS) return 0;
+    return id;
+}
 
 // Device address of the scratch array on the current device.  The name of a __device__
 // array is only a host-side handle, so the address comes from cudaGetSymbolAddress, once
-// per device, with that device current.
+// per device (and again after that device's context was reset), with that device current.
 hstu_status_t noalloc_scratch(void **out)
 {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return HSTU_ERR_CUDA;
     if (dev < 0 || dev >= kMaxDevices) return HSTU_ERR_UNSUPPORTED;
     std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (!g_noalloc_ptr[dev]) {
+    const unsigned long long ctx = current_context_id();
+    if (!g_noalloc_ptr[dev] || ctx == 0 || ctx != g_noalloc_ctx[dev]) {
         void *ptr = nullptr;
         if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr)
             return HSTU_ERR_CUDA;
         g_noalloc_ptr[dev] = ptr;
+        g_noalloc_ctx[dev] = current_context_id();   // the lookup made the context current
     }
     *out = g_noalloc_ptr[dev];
     return HSTU_OK;

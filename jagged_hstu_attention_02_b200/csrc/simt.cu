@@ -94,6 +94,11 @@ __global__ void __launch_bounds__(kThreads)
 
     const int qt = blockIdx.x, b = blockIdx.y, h = blockIdx.z;
     const SeqInfo s = load_seq(p, b, qt == 0 && h == 0 && threadIdx.x == 0);
+    if (qt == 0 && h == 0) {   // rows no block writes: zero Y
+        RowRange rr[3];
+        const int n = skipped_rows(p, b, rr);
+        for (int x = 0; x < n; ++x) zero_rows(y, p.D, rr[x], threadIdx.x, kThreads);
+    }
     const int i0 = qt * kFwdBM;
     if (i0 >= s.L) return;
     const int tid = threadIdx.x, ty = tid / 16, tx = tid % 16;
@@ -331,6 +336,14 @@ __global__ void __launch_bounds__(kThreads)
 
     const int kt = blockIdx.x, b = blockIdx.y, h = blockIdx.z;
     const SeqInfo s = load_seq(p, b, kt == 0 && h == 0 && threadIdx.x == 0);
+    if (kt == 0 && h == 0) {   // rows no block writes: zero dK, dV
+        RowRange rr[3];
+        const int n = skipped_rows(p, b, rr);
+        for (int x = 0; x < n; ++x) {
+            zero_rows(dk, (int64_t)H * dqk, rr[x], threadIdx.x, kThreads);
+            zero_rows(dv_out, (int64_t)H * dv, rr[x], threadIdx.x, kThreads);
+        }
+    }
     const int j0 = kt * kBwdBN;
     if (j0 >= s.L) return;
     const int tid = threadIdx.x, ty = tid / 16, tx = tid % 16;

@@ -61,8 +61,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
 }
 
 // Waits for the phase of `bar` with the given parity to complete.  Returns false if it
-// has not completed within kWaitLimitCycles (the caller then reports and unwinds).
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity)
+// has not completed within `limit` SM clock cycles (the caller then reports and unwinds).
+// Pipeline waits take the launch's limit (kWaitLimitCycles unless a test shortens it); the
+// waits that drain copies and MMAs in flight before a CTA exits always take
+// kWaitLimitCycles.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, long long limit)
 {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
@@ -70,7 +73,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity)
 #pragma unroll 1
         for (int i = 0; i < 4; ++i)
             if (mbar_try_wait(bar, parity)) return true;
-        if (clock64() - t0 > kWaitLimitCycles) return false;
+        if (clock64() - t0 > limit) return false;
     }
 }
 

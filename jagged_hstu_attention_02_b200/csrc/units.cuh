@@ -19,9 +19,9 @@ using sm100::mbar_wait;
 
 constexpr int kUnitRing = 4;
 
-__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity)
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, long long limit)
 {
-    return __all_sync(0xffffffffu, mbar_wait(bar, parity));
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, limit));
 }
 
 // One arrival per warp on `bar` (counted per warp), after the whole warp got here.
@@ -109,7 +109,7 @@ struct UnitFeed {
         ++k;
         if constexpr (ROLE == FEED_PRODUCER) {
             const int64_t u = claim();
-            if (round > 0 && !mbar_wait(&empty[sl], (round - 1) & 1)) {
+            if (round > 0 && !mbar_wait(&empty[sl], (round - 1) & 1, p.wait_limit)) {
                 ok = false;
                 return false;
             }
@@ -118,8 +118,8 @@ struct UnitFeed {
             mbar_arrive(&full[sl]);      // releases the slot's contents
             return u >= 0;
         } else {
-            const bool got = ROLE == FEED_WARP ? warp_wait(&full[sl], round & 1)
-                                               : mbar_wait(&full[sl], round & 1);
+            const bool got = ROLE == FEED_WARP ? warp_wait(&full[sl], round & 1, p.wait_limit)
+                                               : mbar_wait(&full[sl], round & 1, p.wait_limit);
             if (!got) {
                 ok = false;
                 return false;

@@ -23,6 +23,7 @@ DEV_BAD_OFFSETS, DEV_BAD_COUNTS, DEV_SEQ_TOO_LONG, DEV_WAIT_TIMEOUT = 0x1, 0x2, 
 
 EXPORTED = ["hstu_attn_fwd_workspace_size", "hstu_attn_fwd", "hstu_attn_bwd_workspace_size",
             "hstu_attn_bwd", "hstu_attn_read_device_status", "hstu_attn_debug_mask",
+            "hstu_attn_debug_kernel_mask", "hstu_attn_set_wait_test",
             "hstu_attn_time_thresholds", "hstu_attn_set_stage_events", "hstu_status_string",
             "hstu_attn_version"]
 STAGES = {"fwd_attn": 0, "fwd_norm": 1, "bwd_norm": 2, "bwd_attn": 3}
@@ -65,9 +66,12 @@ def lib():
         L.hstu_attn_read_device_status.argtypes = [_VP, _VP, ctypes.POINTER(ctypes.c_int32)]
         L.hstu_attn_debug_mask.argtypes = [P, _VP, _VP, _VP, ctypes.c_int32, ctypes.c_int32, _VP,
                                            _VP]
+        L.hstu_attn_debug_kernel_mask.argtypes = [P, _VP, _VP, _VP] + [ctypes.c_int32] * 5 + [
+            _VP, _VP]
         L.hstu_attn_time_thresholds.argtypes = [ctypes.c_double, ctypes.c_int32,
                                                 ctypes.POINTER(ctypes.c_uint64)]
         L.hstu_attn_set_stage_events.argtypes = [ctypes.c_int32, _VP, _VP]
+        L.hstu_attn_set_wait_test.argtypes = [ctypes.c_int64, ctypes.c_int32]
         L.hstu_status_string.restype = ctypes.c_char_p
         L.hstu_status_string.argtypes = [ctypes.c_int]
         L.hstu_attn_version.restype = ctypes.c_int32
@@ -217,6 +221,23 @@ def debug_mask(params: Params, seq_offsets, num_contextuals, num_targets, seq: i
     return torch.from_numpy(flat[:seq_len * seq_len].reshape(seq_len, seq_len).copy())
 
 
+def debug_kernel_mask(params: Params, seq_offsets, num_contextuals, num_targets, seq: int,
+                      kernel: str, row_begin: int, row_count: int, key_count: int,
+                      stream=None):
+    """[row_count, key_count] bool mask of sequence `seq` as the tensor-core forward
+    (kernel "fwd") or backward ("bwd") decides it, rows from row_begin."""
+    import numpy as np
+    words = row_count * key_count // 32
+    bits = torch.zeros(max(words, 1), dtype=torch.int32, device=seq_offsets.device)
+    _check(lib().hstu_attn_debug_kernel_mask(
+        ctypes.byref(params), _ptr(seq_offsets), _ptr(num_contextuals), _ptr(num_targets), seq,
+        {"fwd": 0, "bwd": 1}[kernel], row_begin, row_count, key_count, _ptr(bits),
+        _stream(stream)), "hstu_attn_debug_kernel_mask")
+    b = bits.cpu().numpy().view("uint32")[:words]
+    flat = ((b[:, None] >> np.arange(32, dtype=np.uint32)[None, :]) & 1).astype(bool).reshape(-1)
+    return torch.from_numpy(flat.reshape(row_count, key_count).copy())
+
+
 def time_thresholds(div: float, nb: int):
     """Host-side threshold table the device compares |dt| against (uint64, nb-1 entries)."""
     arr = (ctypes.c_uint64 * max(nb - 1, 1))()
@@ -230,6 +251,12 @@ def set_stage_events(stage: str, start=None, stop=None):
     sp = None if start is None else ctypes.c_void_p(start.cuda_event)
     ep = None if stop is None else ctypes.c_void_p(stop.cuda_event)
     _check(lib().hstu_attn_set_stage_events(STAGES[stage], sp, ep), "hstu_attn_set_stage_events")
+
+
+def set_wait_test(limit_cycles: int = 0, stall: bool = False):
+    """Test hook: shorten the kernels' pipeline waits and make one of them run out."""
+    _check(lib().hstu_attn_set_wait_test(int(limit_cycles), 1 if stall else 0),
+           "hstu_attn_set_wait_test")
 
 
 def version() -> int:

@@ -114,6 +114,22 @@ int64_t hstu_oracle_mask(int64_t L, int64_t c, int64_t t, int64_t W, uint8_t *ma
     return n;
 }
 
+/* Rows [r0, r0+nrows) x keys [0, ncols) of the same mask, positions past the sequence's end
+ * (>= L) counted invalid; row r - r0 of `mask` has ncols bytes.  Returns the valid count. */
+int64_t hstu_oracle_mask_rows(int64_t L, int64_t c, int64_t t, int64_t W, int64_t r0,
+                              int64_t nrows, int64_t ncols, uint8_t *mask)
+{
+    int64_t n = 0;
+    for (int64_t r = 0; r < nrows; ++r)
+        for (int64_t j = 0; j < ncols; ++j) {
+            int64_t i = r0 + r;
+            int v = i < L && j < L && oracle_valid(i, j, L, c, t, W);
+            mask[r * ncols + j] = (uint8_t)v;
+            n += v;
+        }
+    return n;
+}
+
 typedef struct {
     int64_t B, H, dqk, dv;
     const int64_t *offsets;

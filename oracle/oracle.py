@@ -37,6 +37,8 @@ def lib():
         L.hstu_oracle_mask.argtypes = [_I64, _I64, _I64, _I64, _P_U8]
         common = [_I64, _I64, _I64, _I64, _P_I64, _P_I32, _P_I32, _P_I64, _P_F64, _P_F64,
                   _P_F64, _P_F64, _P_F64, _I64, _P_F64, _I64, _F64, _F64, _I64, _I64, _F64]
+        L.hstu_oracle_mask_rows.restype = _I64
+        L.hstu_oracle_mask_rows.argtypes = [_I64] * 7 + [_P_U8]
         L.hstu_oracle_fwd.restype = ctypes.c_int
         L.hstu_oracle_fwd.argtypes = common + [_P_F64] * 4
         L.hstu_oracle_bwd.restype = ctypes.c_int
@@ -66,6 +68,14 @@ def mask(L: int, c: int = 0, t: int = 0, W: int = 0):
     m = np.zeros((max(L, 1), max(L, 1)), dtype=np.uint8)[:L, :L].copy()
     n = lib().hstu_oracle_mask(L, c, t, W, _ptr(m, ctypes.c_uint8))
     return m, int(n)
+
+
+def mask_rows(L: int, c: int, t: int, W: int, r0: int, nrows: int, ncols: int):
+    """Rows [r0, r0+nrows) x keys [0, ncols) of the mask of one sequence (positions >= L
+    invalid), as a uint8 matrix."""
+    m = np.zeros((nrows, ncols), dtype=np.uint8)
+    lib().hstu_oracle_mask_rows(L, c, t, W, r0, nrows, ncols, _ptr(m, ctypes.c_uint8))
+    return m
 
 
 def num_threads() -> int:

@@ -93,3 +93,18 @@ def test_time_thresholds_match_oracle_fp64_decision(div, nb):
         assert oracle.time_bucket(t, div, nb) >= kk
         if t > 0:
             assert oracle.time_bucket(t - 1, div, nb) < kk
+
+
+def test_test_hooks_validate_their_arguments():
+    lib = ops.lib()
+    assert lib.hstu_attn_set_wait_test(-1, 0) == 1
+    assert lib.hstu_attn_set_wait_test(1000, 2) == 1
+    assert lib.hstu_attn_set_wait_test(0, 0) == 0
+    p = _params()
+    fake = ctypes.c_void_p(16)   # never dereferenced: every call below fails validation first
+    for args in [(0, 2, 0, 4, 128), (0, 0, -1, 4, 128), (0, 0, 0, -4, 128), (0, 0, 0, 4, 100),
+                 (5, 0, 0, 4, 128), (-1, 1, 0, 4, 128)]:
+        seq, kernel, r0, nrows, nkeys = args
+        st = lib.hstu_attn_debug_kernel_mask(ctypes.byref(p), fake, None, None, seq, kernel, r0,
+                                             nrows, nkeys, fake, None)
+        assert st == 1, args

@@ -390,3 +390,16 @@ def test_backward_finite_differences_tiny_workload_shapes():
     b = synth.make_config(0)
     dout = np.random.default_rng(43).standard_normal(b.u.shape)
     _fd_check(b, dout, samples=3)
+
+
+def test_mask_rows_is_the_mask_with_padding_invalid():
+    """The row-range mask equals rows of the full mask, with every position past the end
+    invalid (pinned through the full mask, itself pinned by the golden examples)."""
+    for L, c, t, W in [(300, 4, 20, 50), (129, 32, 32, 0), (7, 0, 7, 0), (1, 1, 0, 3)]:
+        full, _ = oracle.mask(L, c, t, W)
+        pad = (L + 127) // 128 * 128
+        for r0, n in [(0, L), (L // 2, pad - L // 2), (max(L - 3, 0), 10)]:
+            m = oracle.mask_rows(L, c, t, W, r0, n, pad)
+            rows_in = max(min(n, L - r0), 0)
+            assert np.array_equal(m[:rows_in, :L], full[r0:r0 + rows_in])
+            assert not m[rows_in:].any() and not m[:, L:].any()

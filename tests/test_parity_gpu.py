@@ -258,6 +258,42 @@ def test_bad_device_data_is_reported_and_the_context_stays_usable():
     _fwd_check(b, what="after bad data")
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_uncovered_rows_are_zero_and_flagged(dtype):
+    """Offsets that start after row 0 or end before row T, and a sequence skipped for bad
+    counts: the status word says so, the rows no valid sequence covers come out as zeros in
+    out, saved Y, dK and dV, and the other sequences still match the oracle."""
+    lengths = [30, 150, 60, 40]
+    b = synth.make_batch(np.random.default_rng(12), lengths, 2, 64, 64, dtype,
+                         contextuals=[1, 2, 3, 1], targets=[2, 5, 3, 1], rel_bias_len=151,
+                         time_bias_len=128, with_dout=True)
+    dev = ops.batch_to_device(b)
+    offs = b.seq_offsets.copy()
+    offs[0] = 5                   # rows 0..4 uncovered; sequence 0 skipped (does not start at 0)
+    offs[-1] -= 7                 # last sequence ends 7 rows short of T: skipped
+    bad = dict(dev)
+    bad["seq_offsets"] = torch.from_numpy(offs).cuda()
+    bad["num_targets"] = torch.tensor([2, 500, 3, 1], dtype=torch.int32, device="cuda")
+    T = b.total_tokens
+    out, saved = ops.run_fwd(b, bad, training=True)
+    code = ops.read_device_status(ops.fwd.last_workspace)
+    assert code & ops.DEV_BAD_OFFSETS and code & ops.DEV_BAD_COUNTS
+    g = ops.run_bwd(b, saved, dev_tensors=bad)
+    torch.cuda.synchronize()
+    dead = np.zeros(T, bool)
+    dead[:offs[1]] = True                        # rows 0..4 and sequence 0
+    dead[offs[1]:offs[2]] = True                 # sequence 1 (c + t > L)
+    dead[offs[3]:] = True                        # sequence 3 and the 7 rows after it
+    for t_, name in ((out, "out"), (saved.y, "y"), (g[1], "dk"), (g[2], "dv"), (g[0], "dq"),
+                     (g[3], "du")):
+        a = _np(t_).reshape(T, -1)
+        assert np.all(a[dead] == 0), name + ": an uncovered row is not zero"
+    # sequence 2 alone is intact
+    ref = oracle.fwd(sub_batch(b, [2]))
+    rows = rows_of(b, [2])
+    assert_close(_np(out)[rows], ref["out"], dtype, "intact sequence out")
+
+
 # ------------------------------------------------------------------ timestamp orders and ranges
 #
 # The workloads draw ascending timestamps; the kernels exploit ascending order only for
@@ -345,3 +381,137 @@ def test_tile_count_past_the_cache_range():
                          targets=[8, 3, 20], max_attn_len=64, rel_bias_len=65,
                          time_bias_len=128, with_dout=True)
     _fwd_bwd_check(b, "33000-token sequence")
+
+
+# ------------------------------------------------------------------ table-size branches
+#
+# The backward keeps the rel table in shared memory up to 2048 entries and the forward up
+# to 4352; longer tables are read (and the backward's gradient added) in global memory.
+# Sequences of config-2-like lengths with R = N + 1 reach those branches; a window keeps the
+# oracle quick while contextual keys far back still use the high table indices.
+
+def _long_table_batch(seed, lengths, W, H=2):
+    N = int(max(lengths))
+    return synth.make_batch(np.random.default_rng(seed), lengths, H, 128, 128, "bf16",
+                            contextuals=4, targets=64, max_attn_len=W, rel_bias_len=N + 1,
+                            time_bias_len=128, with_dout=True)
+
+
+def test_bwd_parity_rel_table_in_global_memory():
+    b = _long_table_batch(2049, [3100, 4096, 700], W=256)
+    assert b.rel_bias_len > 2048
+    _fwd_bwd_check(b, "R=%d backward" % b.rel_bias_len)
+
+
+def test_fwd_parity_rel_table_in_global_memory():
+    b = _long_table_batch(4353, [4500, 1300], W=300)
+    assert b.rel_bias_len > 4352
+    _fwd_bwd_check(b, "R=%d forward" % b.rel_bias_len)
+
+
+@pytest.mark.parametrize("cfg", [2, 3])
+def test_training_forward_long_workloads_sampled(cfg):
+    """The training forward (A carried as a bf16 hi + lo pair) on the full long-history and
+    windowed batches; out, Y, mean and rstd checked on sampled whole sequences."""
+    b = synth.make_config(cfg)
+    dev = ops.batch_to_device(b)
+    out, saved = ops.run_fwd(b, dev, training=True)
+    torch.cuda.synchronize()
+    assert ops.read_device_status(ops.fwd.last_workspace) == 0
+    L = b.lengths
+    seqs = sorted({int(np.argmin(L)), int(np.argmax(L))})
+    ref = oracle.fwd(sub_batch(b, seqs))
+    rows = rows_of(b, seqs)
+    for got, key in ((out, "out"), (saved.y, "y"), (saved.mean, "mean"), (saved.rstd, "rstd")):
+        assert_close(_np(got)[rows], ref[key], b.dtype, "workload %d training %s" % (cfg, key))
+
+
+# ------------------------------------------------------------------ guard bands
+#
+# Every output (and the workspace) sits inside a larger buffer whose bytes before and after
+# it hold NaN (or 0xFF bytes); after the calls those bands must be untouched: no kernel
+# writes outside the buffers it was given.
+
+_PAD = 4096
+
+
+class _Guarded:
+    def __init__(self):
+        self.bufs = []
+
+    def alloc(self, shape, dtype):
+        n = int(np.prod(shape)) if len(shape) else 1
+        if dtype == torch.uint8:
+            whole = torch.full((2 * _PAD + n,), 0xFF, dtype=dtype, device="cuda")
+        else:
+            whole = torch.full((2 * _PAD + n,), float("nan"), dtype=dtype, device="cuda")
+        self.bufs.append((whole, n))
+        return whole[_PAD:_PAD + n].view(*shape)
+
+    def check(self, what):
+        torch.cuda.synchronize()
+        for whole, n in self.bufs:
+            for band in (whole[:_PAD], whole[_PAD + n:]):
+                if whole.dtype == torch.uint8:
+                    assert bool((band == 0xFF).all()), what + ": a guard band was written"
+                else:
+                    assert bool(torch.isnan(band.float()).all()), what + ": a guard band was written"
+
+
+@pytest.mark.parametrize("case", [c for c in SMALL_CASES if c[0] in
+                                  ("bf16-family", "bf16-window", "f32-full-family",
+                                   "bf16-dqk-ne-dv")], ids=lambda c: c[0])
+def test_outputs_stay_inside_their_buffers(case):
+    name, lengths, H, dqk, dv, dtype, ctx, tgt, W, R, NB = case
+    b = synth.make_batch(np.random.default_rng(77), lengths, H, dqk, dv, dtype,
+                         contextuals=ctx, targets=tgt, max_attn_len=W, rel_bias_len=R,
+                         time_bias_len=NB, with_dout=True)
+    dev = ops.batch_to_device(b)
+    kw = ops.batch_kwargs(b)
+    tdt = dev["q"].dtype
+    T, D = b.u.shape
+    g = _Guarded()
+    p = ops.make_params(dev["q"], dev["v"], dev["seq_offsets"], alpha=b.alpha,
+                        max_seqlen=b.max_seqlen, max_attn_len=b.max_attn_len,
+                        rel_bias=dev["rel_bias"], time_bias=dev["time_bias"])
+    out = g.alloc((T, D), tdt)
+    saved = ops.Saved(g.alloc((T, D), torch.float32), g.alloc((T,), torch.float32),
+                      g.alloc((T,), torch.float32))
+    ws_f = g.alloc((ops.fwd_workspace_size(p),), torch.uint8)
+    args = (dev["q"], dev["k"], dev["v"], dev["u"], dev["seq_offsets"], dev["num_contextuals"],
+            dev["num_targets"], dev["timestamps"], dev["rel_bias"], dev["time_bias"])
+    ops.fwd(*args, out=out, workspace=ws_f, **kw)
+    g.check(name + " inference forward")
+    ops.fwd(*args, training=True, out=out, saved=saved, workspace=ws_f, **kw)
+    g.check(name + " training forward")
+    grads = (g.alloc(tuple(b.q.shape), tdt), g.alloc(tuple(b.k.shape), tdt),
+             g.alloc(tuple(b.v.shape), tdt), g.alloc((T, D), tdt),
+             g.alloc((R,), torch.float32) if R else None,
+             g.alloc((NB,), torch.float32) if NB else None)
+    ws_b = g.alloc((ops.bwd_workspace_size(p),), torch.uint8)
+    ops.bwd(dev["dout"], *args, saved=saved, grads=grads, workspace=ws_b, **kw)
+    g.check(name + " backward")
+    ref = oracle.bwd(b)
+    assert_close(_np(out), oracle.fwd(b)["out"], dtype, name + " guarded out")
+    assert_close(_np(grads[0]), ref["dq"], dtype, name + " guarded dq")
+
+
+# ------------------------------------------------------------------ bounded waits
+
+def test_a_wait_that_runs_out_is_reported_and_the_context_stays_usable():
+    """The MMA issuer of both tensor-core kernels waits on a barrier nothing completes, with
+    a limit of 2e7 cycles (about 10 ms): the wait runs out, HSTU_DEV_WAIT_TIMEOUT is set,
+    every role unwinds, and the next normal calls still match the oracle."""
+    b = synth.make_batch(np.random.default_rng(15), [70, 300, 129], 2, 128, 128, "bf16",
+                         contextuals=[1, 2, 3], targets=[2, 20, 1], rel_bias_len=301,
+                         time_bias_len=128, with_dout=True)
+    dev = ops.batch_to_device(b)
+    try:
+        ops.set_wait_test(20_000_000, stall=True)
+        out, saved = ops.run_fwd(b, dev, training=True)
+        assert ops.read_device_status(ops.fwd.last_workspace) & ops.DEV_WAIT_TIMEOUT
+        ops.run_bwd(b, saved, dev_tensors=dev)
+        assert ops.read_device_status(ops.bwd.last_workspace) & ops.DEV_WAIT_TIMEOUT
+    finally:
+        ops.set_wait_test(0, stall=False)
+    _fwd_bwd_check(b, "after the stall test")
