@@ -1,14 +1,21 @@
-"""Benchmark of the jagged HSTU attention training step (forward + backward) on B200.
+"""Benchmark of jagged HSTU attention on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-One step = one pass of the whole path over one batch of the MovieLens-shaped training
-workload (B=128, H=4, d=128, bf16, Zipf history + 1 contextual + 1..20 candidate tokens,
-time and rel-pos bias, dO ~ N(0,1)): forward with saved activations, then backward.
-Throughput counts valid (unmasked) pairs only: fwd P*H*2*(d_qk+d_v) + bwd P*H*2*(2d_qk+2d_v).
+Headline: the training step on the MovieLens-shaped workload (B=128 per GPU, H=4, d=128,
+bf16, Zipf history + 1 contextual + 1..20 candidate tokens, time and rel-pos bias,
+dO ~ N(0,1)): forward with saved activations, then backward.  One step = one pass of the
+whole path over one batch.  Throughput counts valid (unmasked) pairs only:
+fwd P*H*2*(d_qk+d_v) + bwd P*H*2*(2d_qk+2d_v).
 
-Prints ONE JSON line on rank 0.  Under torchrun each rank runs its own batch (seed + rank),
-no collective on the data path ("scaling": "weak"); timing is the max over ranks.
+Under torchrun the global batch holds N*128 sequences; shard.plan deals them to the ranks
+by longest-processing-time on their pair work, every rank runs with the global max_seqlen,
+and the bias-table gradients are summed with one all-reduce per step ("scaling": "weak":
+the work per GPU stays fixed as N grows).  Timing is the max over ranks.
+
+On one GPU the line also carries one block per inference-forward workload (long history,
+windowed, MovieLens-shaped), each timed over >= 50 L2-flushed calls with its own roofline,
+clocks and CPU baseline.  Prints ONE JSON line on rank 0.
 """
 from __future__ import annotations
 
@@ -29,15 +36,19 @@ from jagged_hstu_attention_02_b200 import accounting, synth  # noqa: E402
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 << 20
 WORKLOAD_CFG = 4          # MovieLens-shaped inputs + upstream gradient
-SECONDARY_CFG = 2         # long-history forward (tensor-core regime)
+# inference-forward blocks: workload -> (block name, roofline that bounds its attention kernel)
+FWD_BLOCKS = {2: ("long_history_fwd", "tensor"), 3: ("windowed_fwd", "tensor"),
+              1: ("movielens_fwd", "hbm")}
 
 
 # DRAM traffic per launch of a kernel, from an ncu capture summarised under profiles/; used
 # only while the kernel's sources hash to the value recorded with the capture.
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 KERNEL_SOURCES = {
-    "bwd_attn": ["bwd_sm100.cu", "bias.cuh", "common.cuh", "sm100.cuh", "units.cuh"],
-    "fwd_attn": ["fwd_sm100.cu", "bias.cuh", "common.cuh", "sm100.cuh", "units.cuh"],
+    "bwd_attn": ["bwd_sm100.cu", "bias.cuh", "common.cuh", "sm100.cuh", "tiles.cuh",
+                 "units.cuh"],
+    "fwd_attn": ["fwd_sm100.cu", "bias.cuh", "common.cuh", "sm100.cuh", "tiles.cuh",
+                 "units.cuh"],
 }
 
 
@@ -56,8 +67,8 @@ def recorded_traffic(stage, workload):
     if not os.path.exists(TRAFFIC_FILE):
         return None, "no capture recorded"
     with open(TRAFFIC_FILE) as f:
-        rec = json.load(f).get(stage)
-    if not rec or rec.get("workload") != workload:
+        rec = json.load(f).get("%s@%d" % (stage, workload))
+    if not rec:
         return None, "no capture of this workload"
     if rec.get("sources_sha") != sources_sha(stage):
         return None, "kernel changed since the capture"
@@ -151,6 +162,19 @@ def stage_timer(ops, torch, stages):
     return evs
 
 
+def headline_batch(world, rank):
+    """This rank's share of the global training batch: N*128 MovieLens-shaped sequences dealt
+    by shard.plan, all with the global max_seqlen (and rel table of N+1 entries)."""
+    from jagged_hstu_attention_02_b200 import shard
+
+    g = synth.make_config(WORKLOAD_CFG, batch=128 * world)
+    if world == 1:
+        return g, g
+    seqs = shard.plan(g.seq_offsets, world, g.num_contextuals, g.num_targets,
+                      g.max_attn_len)[rank]
+    return synth.sub_batch(g, seqs), g
+
+
 def run_ours(args, world, rank, local):
     import torch
     from jagged_hstu_attention_02_b200 import ops
@@ -162,9 +186,11 @@ def run_ours(args, world, rank, local):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     peaks, peak_kind = load_peaks()
 
-    b = synth.make_config(WORKLOAD_CFG, seed=synth.BASE_SEED + 1 + 1000 * rank)
+    b, gb = headline_batch(world, rank)
     P = accounting.valid_pairs(b)
     flops = accounting.fwd_flops(b, P) + accounting.bwd_flops(b, P)
+    P_all = accounting.valid_pairs(gb)
+    flops_all = accounting.fwd_flops(gb, P_all) + accounting.bwd_flops(gb, P_all)
     tokens = b.total_tokens
     dev = ops.batch_to_device(b)
     kw = ops.batch_kwargs(b)
@@ -209,6 +235,10 @@ def run_ours(args, world, rank, local):
         ops.set_stage_events(s)
     avg = {s: sum(v) / len(v) for s, v in stage_ms.items()}
     dom = max(avg, key=avg.get)
+    if world > 1:   # every rank times the same stage (the graph below depends on it)
+        t = torch.tensor([stages.index(dom)], device="cuda")
+        torch.distributed.broadcast(t, 0)
+        dom = stages[int(t.item())]
 
     # the measured steps replay one CUDA graph of the step's library calls (the table-grad
     # all-reduce of a sharded step stays outside it), with no events between its kernels:
@@ -278,34 +308,27 @@ def run_ours(args, world, rank, local):
         t = torch.tensor([ms], device="cuda")
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         ms = float(t.item())
-    value = world * flops / (ms * 1e-3) / 1e12
+    value = flops_all / (ms * 1e-3) / 1e12
 
-    # roofline of the dominant kernel stage, timed inside the measured steps
+    # roofline of the dominant kernel stage, timed inside the measured steps, on its own
+    # algorithmic bytes and FLOPs
     avg[dom] = sum(dom_ms) / len(dom_ms)
-    dom_bytes = {"fwd_attn": accounting.fwd_bytes(b, training=True),
-                 "fwd_norm": b.total_tokens * b.num_heads * b.d_v * (4 + 2 + 2) + 8 * tokens,
-                 "bwd_norm": b.total_tokens * b.num_heads * b.d_v * (2 + 2 + 4 + 2 + 4) + 8 * tokens,
-                 "bwd_attn": accounting.bwd_bytes(b)}[dom]
-    dom_flops = {"fwd_attn": accounting.fwd_flops(b, P), "bwd_attn": accounting.bwd_flops(b, P)}
-    hbm_peak = peaks["hbm_gbs"]
-    achieved = dom_bytes / (avg[dom] * 1e-3) / 1e9
-    traffic, traffic_note = recorded_traffic(dom, WORKLOAD_CFG)
-    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak,
-                "unit": "GB/s", "frac": round(achieved / hbm_peak, 4), "traffic": traffic,
-                "traffic_note": traffic_note, "algorithmic_bytes": dom_bytes,
-                "kernel_stage": dom, "kernel_ms": round(avg[dom], 4),
-                "peak_source": peak_kind, "stage_ms": {s: round(v, 4) for s, v in avg.items()},
-                "stage_ms_note": "kernel_ms from replays of the step graph with the kernel's two "
-                                 "events inside; the other stages from eager steps with events "
-                                 "between all kernels"}
-    if dom in dom_flops:
-        roofline["tflops"] = round(dom_flops[dom] / (avg[dom] * 1e-3) / 1e12, 2)
+    roofline = kernel_roofline(b, dom, avg[dom], P, peaks, peak_kind, WORKLOAD_CFG,
+                               training=True)
+    roofline["stage_ms"] = {s: round(v, 4) for s, v in avg.items()}
+    roofline["stage_ms_note"] = ("kernel_ms from replays of the step graph with the kernel's "
+                                 "two events inside; the other stages from eager steps with "
+                                 "events between all kernels")
 
     # end to end through the public API with host buffers (pinned), copies inside the region
-    e2e = measure_e2e(args, b, ops, torch, kw, flops, world)
+    e2e = measure_e2e(args, b, ops, torch, kw, flops, world, flops_all)
 
-    secondary = measure_secondary(ops, torch, peaks, rank) if rank == 0 and not args.quick else None
-    cpu = cpu_baseline(b) if (rank == 0 and world == 1 and not args.no_cpu) else None
+    blocks = {}
+    if world == 1 and not args.quick:
+        for cfg in FWD_BLOCKS:
+            blocks[FWD_BLOCKS[cfg][0]] = measure_fwd_block(ops, torch, peaks, peak_kind, cfg,
+                                                           args, with_cpu=not args.no_cpu)
+    cpu = cpu_baseline_train(b) if (rank == 0 and world == 1 and not args.no_cpu) else None
     if world > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
@@ -316,17 +339,20 @@ def run_ours(args, world, rank, local):
         "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "tokens_per_s": round(world * tokens / (ms * 1e-3), 1),
+        "tokens_per_s": round(gb.total_tokens / (ms * 1e-3), 1),
         "pct_bf16_peak": round(100 * value / world / peaks["bf16_tflops"], 3),
-        "config": {"workload": synth.WORKLOADS[WORKLOAD_CFG], "global_batch": b.batch * world,
-                   "tokens_per_gpu": tokens, "valid_pairs_per_gpu": P, "flops_per_step": flops,
-                   "max_seqlen": b.max_seqlen, "parallelism": "dp%d" % world,
+        "config": {"workload": synth.WORKLOADS[WORKLOAD_CFG], "global_batch": gb.batch,
+                   "tokens_per_gpu": tokens, "tokens_global": gb.total_tokens,
+                   "valid_pairs_global": P_all, "flops_per_step_global": flops_all,
+                   "max_seqlen": gb.max_seqlen, "parallelism": "dp%d" % world,
+                   "sharding": "shard.plan (LPT on valid pairs) over the global batch" if world > 1
+                   else "one GPU, whole batch",
                    "l2": "flushed between steps (256 MB write), flush outside per-step events",
                    "launch": "each step replays one CUDA graph of its fwd and bwd library calls",
                    "wall_s_region": round(wall_region, 3)},
         "roofline": roofline, "e2e": e2e, "clocks": clk,
         "gpu_launches": args.steps * LAUNCHES_PER_STEP,
-        "cpu_baseline": cpu, "secondary": secondary,
+        "cpu_baseline": cpu, "workloads": blocks,
     }
     print(json.dumps(line), flush=True)
 
@@ -334,9 +360,40 @@ def run_ours(args, world, rank, local):
 # kernels of ours launched per step: fwd attention, fwd LayerNorm+gating, bwd LayerNorm+gating,
 # bwd attention, dQ conversion (memsets are not kernels of ours)
 LAUNCHES_PER_STEP = 5
+LAUNCHES_PER_FWD = 2
 
 
-def measure_e2e(args, b, ops, torch, kw, flops, world):
+def kernel_roofline(b, stage, kms, P, peaks, peak_kind, workload, training, bound=None):
+    """Roofline of one kernel stage from its own algorithmic bytes and valid-pair FLOPs:
+    HBM-bound unless its arithmetic intensity is above the ridge point (or `bound` says)."""
+    byts = {"fwd_attn": accounting.fwd_attn_bytes(b, training=training),
+            "fwd_norm": accounting.fwd_norm_bytes(b, training=training),
+            "bwd_norm": accounting.bwd_norm_bytes(b),
+            "bwd_attn": accounting.bwd_attn_bytes(b)}[stage]
+    fl = {"fwd_attn": accounting.fwd_flops(b, P), "bwd_attn": accounting.bwd_flops(b, P)}.get(
+        stage, 0)
+    gbs = byts / (kms * 1e-3) / 1e9
+    tfs = fl / (kms * 1e-3) / 1e12
+    hbm, tc = peaks["hbm_gbs"], peaks["bf16_tflops"]
+    ridge = tc * 1e12 / (hbm * 1e9)
+    if bound is None:
+        bound = "tensor" if fl and fl / byts > ridge else "hbm"
+    traffic, traffic_note = recorded_traffic(stage, workload)
+    r = {"bound": bound}
+    if bound == "tensor":
+        r.update(achieved=round(tfs, 2), peak=tc, unit="TFLOP/s", frac=round(tfs / tc, 4),
+                 peak_note="bf16_tflops (burst: the kernel is timed alone)")
+    else:
+        r.update(achieved=round(gbs, 1), peak=hbm, unit="GB/s", frac=round(gbs / hbm, 4))
+    r.update(traffic=traffic, traffic_note=traffic_note, algorithmic_bytes=byts,
+             algorithmic_flops=fl, kernel_stage=stage, kernel_ms=round(kms, 4),
+             peak_source=peak_kind, hbm_frac=round(gbs / hbm, 4),
+             tensor_frac=round(tfs / tc, 4) if fl else None,
+             intensity_flop_per_byte=round(fl / byts, 2), ridge_flop_per_byte=round(ridge, 1))
+    return r
+
+
+def measure_e2e(args, b, ops, torch, kw, flops, world, flops_all):
     """Training steps through the public API with every step's inputs copied in from pinned
     host memory and its results (O, dQ, dK, dV, dU, table gradients) read back.  As a
     training loop would, the copies run on their own streams into and out of double
@@ -397,6 +454,9 @@ def measure_e2e(args, b, ops, torch, kw, flops, world):
                 ops.bwd(d["dout"], d["q"], d["k"], d["v"], d["u"], d["seq_offsets"],
                         d["num_contextuals"], d["num_targets"], d["timestamps"], d["rel_bias"],
                         d["time_bias"], saved=saveds[k], grads=gradss[k], **kw)
+                if world > 1:
+                    torch.distributed.all_reduce(gradss[k][4])
+                    torch.distributed.all_reduce(gradss[k][5])
                 comp_done[k].record(s_comp)
             with torch.cuda.stream(s_out):          # step i's results back to the host
                 s_out.wait_event(comp_done[k])
@@ -408,6 +468,8 @@ def measure_e2e(args, b, ops, torch, kw, flops, world):
     e0.record()
     run(max(args.warmup, 3), e0)
     torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
     e0.record()
     run(args.steps, e0)
     for st in (s_in, s_comp, s_out):
@@ -415,90 +477,161 @@ def measure_e2e(args, b, ops, torch, kw, flops, world):
     e1.record()
     e1.synchronize()
     ms = e0.elapsed_time(e1) / args.steps
-    return {"value": round(world * flops / (ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+    if world > 1:
+        t = torch.tensor([ms], device="cuda")
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    return {"value": round(flops_all / (ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
             "ms_per_step": round(ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "overlap": "inputs of step i+1 and results of step i-1 copied while step i runs"}
 
 
-def measure_secondary(ops, torch, peaks, rank):
-    """Long-history forward (the tensor-core regime): valid-pair TFLOP/s and % of bf16 peak."""
-    b = synth.make_config(SECONDARY_CFG)
+def measure_fwd_block(ops, torch, peaks, peak_kind, cfg, args, with_cpu=True):
+    """One inference-forward workload: >= 50 L2-flushed calls through the API (CUDA events
+    around each call, the flush outside them), then as many again with the library's stage
+    events around the attention kernel; median times; clocks sampled during the first set."""
+    name, bound = FWD_BLOCKS[cfg]
+    iters = max(50, args.steps)
+    b = synth.make_config(cfg)
     P = accounting.valid_pairs(b)
     fl = accounting.fwd_flops(b, P)
     dev = ops.batch_to_device(b)
     out = ops.run_fwd(b, dev)
     ws = ops.fwd.last_workspace
     kw = ops.batch_kwargs(b)
-    evs = stage_timer(ops, torch, ["fwd_attn"])
-    times, kt = [], []
-    for it in range(8):
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+
+    def call():
         ops.fwd(dev["q"], dev["k"], dev["v"], dev["u"], dev["seq_offsets"],
                 dev["num_contextuals"], dev["num_targets"], dev["timestamps"], dev["rel_bias"],
                 dev["time_bias"], out=out, workspace=ws, **kw)
+
+    for _ in range(max(args.warmup, 3)):
+        flush.fill_(1.0)
+        call()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    times = []
+    for _ in range(iters):
+        flush.fill_(1.0)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        call()
         e1.record()
         e1.synchronize()
-        if it >= 3:
-            times.append(e0.elapsed_time(e1))
-            kt.append(evs["fwd_attn"][0].elapsed_time(evs["fwd_attn"][1]))
+        times.append(e0.elapsed_time(e1))
+    clk = clocks.stop()
+    evs = stage_timer(ops, torch, ["fwd_attn"])
+    kt = []
+    for _ in range(iters):
+        flush.fill_(1.0)
+        call()
+        torch.cuda.synchronize()
+        kt.append(evs["fwd_attn"][0].elapsed_time(evs["fwd_attn"][1]))
     ops.set_stage_events("fwd_attn")
-    ms = sum(times) / len(times)
-    kms = sum(kt) / len(kt)
-    tf = fl / (ms * 1e-3) / 1e12
-    ktf = fl / (kms * 1e-3) / 1e12
-    return {"workload": synth.WORKLOADS[SECONDARY_CFG], "metric": "fwd TFLOP/s (valid pairs)",
-            "value": round(tf, 2), "ms": round(ms, 4), "attn_kernel_ms": round(kms, 4),
-            "attn_kernel_tflops": round(ktf, 2),
-            "frac_of_bf16_peak": round(ktf / peaks["bf16_tflops"], 4),
-            "tokens_per_s": round(b.total_tokens / (ms * 1e-3), 1), "valid_pairs": P}
+    assert ops.read_device_status(ws) == 0
+    ms = statistics.median(times)
+    kms = statistics.median(kt)
+    blk = {"workload": synth.WORKLOADS[cfg], "metric": "fwd TFLOP/s (valid pairs)",
+           "value": round(fl / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+           "ms_per_call": round(ms, 4), "iters": iters, "timing": "median of CUDA-event times",
+           "l2": "flushed before every call (256 MB write, outside the events)",
+           "tokens_per_s": round(b.total_tokens / (ms * 1e-3), 1), "tokens": b.total_tokens,
+           "valid_pairs": P, "flops_per_call": fl, "max_seqlen": b.max_seqlen,
+           "roofline": kernel_roofline(b, "fwd_attn", kms, P, peaks, peak_kind, cfg,
+                                       training=False, bound=bound),
+           "clocks": clk, "gpu_launches": iters * LAUNCHES_PER_FWD}
+    if cfg == 3:
+        visited = accounting.tiles_with_pairs(b)
+        blk["tile_skip_efficiency"] = round(P / (visited * 128 * 128), 4)
+        blk["tile_skip_note"] = ("valid pairs / pairs of the 128x128 tiles visited (tiles "
+                                 "holding a valid pair: %d of %d)" % (
+                                     visited, int(sum(((L + 127) // 128) ** 2 for L in b.lengths))))
+    if with_cpu:
+        blk["cpu_baseline"] = cpu_baseline_fwd(b)
+    return blk
 
 
-def cpu_baseline(b, target_s=15.0):
-    """The fp64 oracle, as it stands, on a bounded sample of the workload's sequences."""
+def _timed_sample(b, run, target_s):
+    """Times `run` (the oracle, parallel over sequences) on a sample of b's first sequences:
+    one sequence first; if that is quick, as many sequences as the oracle has threads, then
+    doubling until a run takes target_s / 4 (or the whole batch).  Returns (sequences,
+    sub-batch, seconds, threads busy)."""
     from oracle import oracle
 
-    order = list(range(b.batch))
-    n = max(1, b.batch // 8)
+    threads = oracle.num_threads()
+    n = 1
     while True:
-        sb = synth.sub_batch(b, order[:n])
+        sb = synth.sub_batch(b, list(range(n)))
         t0 = time.perf_counter()
-        oracle.fwd(sb)
-        oracle.bwd(sb)
+        run(sb)
         el = time.perf_counter() - t0
         if el > target_s / 4 or n >= b.batch:
-            break
-        n = min(b.batch, n * 2)
+            return n, sb, el, min(n, threads)
+        n = min(b.batch, threads if n < threads else n * 2)
+
+
+def cpu_baseline_train(b, target_s=15.0):
+    """The fp64 oracle, as it stands, on a bounded sample of the training workload."""
+    from oracle import oracle
+
+    def run(sb):
+        oracle.fwd(sb)
+        oracle.bwd(sb)
+
+    n, sb, el, cores = _timed_sample(b, run, target_s)
     P = accounting.valid_pairs(sb)
     fl = accounting.fwd_flops(sb, P) + accounting.bwd_flops(sb, P)
-    return {"value": round(fl / el / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
+    return {"value": round(fl / el / 1e12, 6), "unit": "TFLOP/s", "cores": cores,
             "kind": "oracle", "seconds": round(el, 3),
-            "sample": "first %d of %d sequences (%d tokens), fwd+bwd in fp64" %
-                      (n, b.batch, sb.total_tokens)}
+            "sample": "first %d of %d sequences (%d tokens), fwd+bwd in fp64, one thread "
+                      "per sequence" % (n, b.batch, sb.total_tokens)}
+
+
+def cpu_baseline_fwd(b, target_s=12.0):
+    """The fp64 oracle forward, as it stands, on a bounded sample of a forward workload."""
+    from oracle import oracle
+
+    n, sb, el, cores = _timed_sample(b, oracle.fwd, target_s)
+    P = accounting.valid_pairs(sb)
+    fl = accounting.fwd_flops(sb, P)
+    return {"value": round(fl / el / 1e12, 6), "unit": "TFLOP/s", "cores": cores,
+            "kind": "oracle", "seconds": round(el, 3),
+            "sample": "first %d of %d sequences (%d tokens), forward in fp64, one thread "
+                      "per sequence" % (n, b.batch, sb.total_tokens)}
 
 
 def run_reference(args, world, rank):
-    """The oracle timed on the host cores as the reference arm (rank 0 only)."""
+    """The oracle timed on the host cores as the reference arm (rank 0 only): every step is
+    the fp64 forward + backward of all sequences of the training workload."""
     if rank != 0:
         return
     from oracle import oracle
 
-    b = synth.make_config(WORKLOAD_CFG)
-    n = max(1, b.batch // 16)
-    sb = synth.sub_batch(b, list(range(n)))
-    P = accounting.valid_pairs(sb)
-    fl = accounting.fwd_flops(sb, P) + accounting.bwd_flops(sb, P)
-    for _ in range(min(args.warmup, 1)):
-        oracle.fwd(sb)
-        oracle.bwd(sb)
+    full = synth.make_config(WORKLOAD_CFG)
+    t0 = time.perf_counter()
+    oracle.fwd(full)                 # warm-up step on the whole batch, which also sizes it
+    oracle.bwd(full)
+    el_full = time.perf_counter() - t0
+    # keep the run within about two minutes: when K whole-batch steps would take longer,
+    # every step takes every k-th sequence (the length mix kept), at least 4 per core
+    k = 1
+    while (args.steps * el_full / (k * 2) > 120.0 and
+           full.batch // (k * 2) >= 4 * oracle.num_threads()):
+        k *= 2
+    b = full if k == 1 else synth.sub_batch(full, list(range(0, full.batch, k)))
+    P = accounting.valid_pairs(b)
+    fl = accounting.fwd_flops(b, P) + accounting.bwd_flops(b, P)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle.fwd(sb)
-        oracle.bwd(sb)
+        oracle.fwd(b)
+        oracle.bwd(b)
     el = (time.perf_counter() - t0) / args.steps
     v = fl / el / 1e12
-    sample = "first %d of %d sequences per step (%d tokens), fwd+bwd in fp64" % (
-        n, b.batch, sb.total_tokens)
+    sample = ("%s %d of %d sequences per step (%d tokens), fwd+bwd in fp64" %
+              ("all" if k == 1 else "every %d-th sequence:" % k, b.batch, full.batch,
+               b.total_tokens))
     line = {"impl": "reference",
             "metric": "jagged HSTU attn fwd+bwd TFLOP/s (valid pairs) on 1 B200",
             "value": round(v, 6), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -519,15 +652,18 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--quick", action="store_true", help="skip the long-history secondary line")
-    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
-    ap.add_argument("--secondary-only", action="store_true",
-                    help="only the long-history forward line (for profiling its kernel)")
+    ap.add_argument("--quick", action="store_true", help="skip the inference-forward blocks")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baselines")
+    ap.add_argument("--fwd-only", type=int, default=None, metavar="WORKLOAD",
+                    help="only the inference-forward block of this workload (1, 2 or 3), "
+                         "without CPU baseline (for profiling its kernel)")
     args = ap.parse_args()
-    if args.secondary_only:
+    if args.fwd_only is not None:
         import torch
         from jagged_hstu_attention_02_b200 import ops
-        print(json.dumps(measure_secondary(ops, torch, load_peaks()[0], 0)), flush=True)
+        peaks, kind = load_peaks()
+        print(json.dumps(measure_fwd_block(ops, torch, peaks, kind, args.fwd_only, args,
+                                           with_cpu=False)), flush=True)
         return
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3

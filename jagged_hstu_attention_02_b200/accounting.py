@@ -115,3 +115,102 @@ def bwd_bytes(batch) -> int:
     n += 8 * (B + 1) + 4 * B * 2
     n += 2 * 4 * (batch.rel_bias_len + batch.time_bias_len)
     return n
+
+
+# ------------------------------------------------------------------ per-kernel bytes
+#
+# Algorithmic HBM bytes of each kernel of the path: what it must read and write at least
+# once, whatever its tiling.  Bias tables, per-sequence counts and offsets are counted with
+# the attention kernels.
+
+def _meta_bytes(batch) -> int:
+    B = batch.batch
+    return 8 * (B + 1) + 4 * B * 2 + 4 * (batch.rel_bias_len + batch.time_bias_len)
+
+
+def _ts_bytes(batch) -> int:
+    return 8 * batch.total_tokens if batch.time_bias_len > 0 else 0
+
+
+def fwd_attn_bytes(batch, training: bool = False, fused_norm: bool = False) -> int:
+    """Forward attention kernel: read Q, K, V (+ timestamps, metadata, tables); write Y in
+    fp32.  With the LayerNorm and U gating fused into it, also read U and write O, and write
+    Y only when training (plus mean and rstd)."""
+    T, H, s = batch.total_tokens, batch.num_heads, elem_size(batch.dtype)
+    D = H * batch.d_v
+    n = T * H * (2 * batch.d_qk + batch.d_v) * s + _ts_bytes(batch) + _meta_bytes(batch)
+    if fused_norm:
+        n += 2 * T * D * s                       # U read, O written
+        if training:
+            n += 4 * T * D + 8 * T               # Y, mean, rstd
+    else:
+        n += 4 * T * D                           # Y
+    return n
+
+
+def fwd_norm_bytes(batch, training: bool = False) -> int:
+    """Separate LayerNorm + gating kernel: read Y (fp32) and U, write O (+ mean, rstd)."""
+    T, s = batch.total_tokens, elem_size(batch.dtype)
+    D = batch.num_heads * batch.d_v
+    return T * D * (4 + 2 * s) + (8 * T if training else 0)
+
+
+def bwd_norm_bytes(batch) -> int:
+    """LayerNorm + gating backward: read dO, U, Y (fp32), mean, rstd; write dU and dY (fp32)."""
+    T, s = batch.total_tokens, elem_size(batch.dtype)
+    D = batch.num_heads * batch.d_v
+    return T * D * (3 * s + 4 + 4) + 8 * T
+
+
+def bwd_attn_bytes(batch) -> int:
+    """Backward attention kernel: read Q, K, V, dY (fp32) (+ timestamps, metadata, tables);
+    write dQ, dK, dV and the table gradients."""
+    T, H, s = batch.total_tokens, batch.num_heads, elem_size(batch.dtype)
+    D = H * batch.d_v
+    n = 2 * T * H * (2 * batch.d_qk + batch.d_v) * s     # Q, K, V read; dQ, dK, dV written
+    n += 4 * T * D                                        # dY
+    n += _ts_bytes(batch) + _meta_bytes(batch) + 4 * (batch.rel_bias_len + batch.time_bias_len)
+    return n
+
+
+# ------------------------------------------------------------------ visited tiles
+
+def tiles_with_pairs_seq(L: int, c: int = 0, t: int = 0, W: int = 0, tile: int = 128) -> int:
+    """(query tile, key tile) pairs of one sequence that hold at least one valid pair: the
+    tiles a kernel that skips empty tiles must visit.  Per query tile, the union of its
+    rows' valid key ranges: the contextual prefix (every row), the history rows' causal
+    (windowed) ranges, the candidate rows' history range and their own positions."""
+    if L <= 0:
+        return 0
+    E = L - t
+    nt = (L + tile - 1) // tile
+    total = 0
+    for qt in range(nt):
+        i0, i1 = qt * tile, min(qt * tile + tile, L) - 1
+        keys = set()
+
+        def add(a, b):
+            if a <= b:
+                keys.update(range(a // tile, b // tile + 1))
+
+        if c > 0:
+            add(0, c - 1)                                     # contextual keys / prefix rows
+        ra, rb = max(i0, c), min(i1, E - 1)                   # history rows
+        if ra <= rb:
+            add(max(c, ra - W) if W > 0 else c, rb)
+        ca, cb = max(i0, E), i1                               # candidate rows
+        if ca <= cb:
+            if E > 0:
+                add(max(c, E - 1 - W) if W > 0 else c, E - 1)
+            add(ca, cb)                                       # themselves
+        total += len(keys)
+    return total
+
+
+def tiles_with_pairs(batch, tile: int = 128) -> int:
+    L = np.diff(batch.seq_offsets)
+    B = len(L)
+    c = batch.num_contextuals if batch.num_contextuals is not None else np.zeros(B, np.int32)
+    t = batch.num_targets if batch.num_targets is not None else np.zeros(B, np.int32)
+    return int(sum(tiles_with_pairs_seq(int(L[b]), int(c[b]), int(t[b]),
+                                        int(batch.max_attn_len), tile) for b in range(B)))

@@ -159,17 +159,21 @@ WORKLOADS = {
 }
 
 
-def make_config(cfg: int, seed: Optional[int] = None) -> Batch:
-    """The five workloads, each drawn from default_rng(1234 + cfg) unless `seed` is given."""
+def make_config(cfg: int, seed: Optional[int] = None, batch: Optional[int] = None) -> Batch:
+    """The five workloads, each drawn from default_rng(1234 + cfg) unless `seed` is given.
+    `batch` changes the number of sequences of the MovieLens-shaped workloads (1 and 4),
+    e.g. to draw the global batch of a data-parallel run (128 per GPU)."""
     if seed is None:
         seed = BASE_SEED + (1 if cfg == 4 else cfg)
+    if batch is not None and cfg not in (1, 4):
+        raise ValueError("only the MovieLens-shaped workloads take a batch size")
     rng = np.random.default_rng(seed)
     if cfg == 0:
         lengths = [10, 100, 1000]
         return make_batch(rng, lengths, 2, 32, 32, "f32", rel_bias_len=1001,
                           max_seqlen=1000, name=WORKLOADS[0])
     if cfg in (1, 4):
-        B = 128
+        B = 128 if batch is None else int(batch)
         hist = np.clip(rng.zipf(1.2, size=B), 8, 200).astype(np.int64)
         tgt = rng.integers(1, 21, size=B).astype(np.int32)
         lengths = 1 + hist + tgt

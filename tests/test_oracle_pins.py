@@ -403,3 +403,16 @@ def test_mask_rows_is_the_mask_with_padding_invalid():
             rows_in = max(min(n, L - r0), 0)
             assert np.array_equal(m[:rows_in, :L], full[r0:r0 + rows_in])
             assert not m[rows_in:].any() and not m[:, L:].any()
+
+
+@pytest.mark.parametrize("L,c,t,W", [(300, 4, 20, 50), (129, 32, 32, 0), (7, 0, 7, 0),
+                                     (1, 1, 0, 3), (1000, 100, 200, 129), (513, 0, 0, 0),
+                                     (700, 8, 128, 1024), (260, 1, 5, 1), (64, 0, 64, 0)])
+def test_visited_tile_count_is_the_tiles_holding_a_valid_pair(L, c, t, W):
+    """The accounting's tile count (used for the tile-skip efficiency) equals a brute-force
+    count of the 128 x 128 tiles of the oracle mask that hold a valid pair."""
+    m, _ = oracle.mask(L, c, t, W)
+    nt = (L + 127) // 128
+    brute = sum(1 for a in range(nt) for b in range(nt)
+                if m[a * 128:(a + 1) * 128, b * 128:(b + 1) * 128].any())
+    assert accounting.tiles_with_pairs_seq(L, c, t, W) == brute
