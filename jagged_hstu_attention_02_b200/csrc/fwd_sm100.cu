@@ -50,14 +50,16 @@ constexpr int BM = 128, BN = 128, QW = 32;   // QW: key columns per epilogue war
 static_assert(BM == kTile && BN == kTile && QW == kBlk, "tile shapes of tiles.cuh");
 constexpr int kEpiWarps = 16;                  // four warpgroups
 constexpr int kTcThreads = 128 + 32 * kEpiWarps;
-constexpr int kRelSmemMax = 4352;   // covers N up to 4351 (R = N + 1)
+constexpr int kRelSmemMax = 4352;   // words of the shared rel table region
+// Inference: the rel table is held as bf16 key pairs with kRelGuard entries on both sides
+// (see fwd_quarter_inf); it fits in shared memory for R up to kRelSmemMax - 2 kRelGuard.
+constexpr int kRelGuard = 32;
+constexpr int kRelPairMax = kRelSmemMax - 2 * kRelGuard;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kBlockBytes = 128 * 128;   // one 128-row x 64-element bf16 swizzle block
 constexpr uint32_t kPCol = 256;          // TMEM columns of A (packed bf16)
 constexpr uint32_t kOCol = 384;          // TMEM columns of the output accumulator
 constexpr int KST = 2, VST = 2, QST = 2; // K, V and Q stages
-// mean relative loss of cutting an fp32 to bf16 (dropping 16 bits), ~0.72 * 2^-8
-constexpr float kTruncBump = 1.0028f;
 
 enum Bar { Q_FULL = 0, Q_EMPTY = 2, K_FULL = 4, K_EMPTY = 6, V_FULL = 8, V_EMPTY = 10,
            S_FULL = 12, S_FREE = 14, P_FULL = 16, P_FREE = 18, META_FULL = 20, EPI_DONE = 22,
@@ -125,6 +127,8 @@ struct FwdEpi {
     const int64_t *tk64;       // and absolute
     const float *relp;         // rel table (relp * rel_sc = half bias)
     float rel_sc;
+    const uint32_t *relp2;     // inference: bf16 pair table, relp2[x] = {rel[x], rel[x-1]} / 2
+    const float *relg;         // inference, clamped blocks: the fp32 table (R >= 1 entries)
     int rbase, R;              // rel index of key c: rbase - c (clamped unless RD)
     float half_alpha, alpha;
     const float *tbh;          // half time-bias table
@@ -218,6 +222,98 @@ __device__ __forceinline__ void fwd_quarter(const FwdEpi &e, const HalfTime &ht,
     }
 }
 
+__device__ __forceinline__ uint32_t add_bf16x2(uint32_t a, uint32_t b)
+{
+    uint32_t d;
+    asm("add.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+// Inference: 8 keys (cb .. cb+7) of one row in packed bf16 pairs (key c in the low half,
+// c + 1 in the high half).  With the half bias b/2 and h = (alpha s + b) / 2:
+// SiLU(2h) / 2 = h + h tanh(h), computed as fma(h, tanh(h), h); every conversion rounds to
+// nearest even.  s holds the 8 keys' scores (fp32 bits), a receives the 4 A columns.
+template <int TM, bool RD, bool FULL>
+__device__ __forceinline__ void inf_chunk(const FwdEpi &e, const HalfTime &ht, uint32_t vmask,
+                                          int cb, const uint32_t (&s)[8], uint32_t ha2,
+                                          uint32_t tlo2, uint32_t thi2, uint32_t a1,
+                                          uint32_t span, uint32_t (&a)[4])
+{
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const int c = cb + 2 * q;
+        uint32_t r2;
+        if (RD) {
+            r2 = e.relp2[e.rbase - c];           // guard-banded: no clamp needed here
+        } else {
+            int x0 = e.rbase - c, x1 = x0 - 1;
+            x0 = x0 < 0 ? 0 : (x0 > e.R - 1 ? e.R - 1 : x0);
+            x1 = x1 < 0 ? 0 : (x1 > e.R - 1 ? e.R - 1 : x1);
+            r2 = pack_bf16x2(0.5f * e.relg[x0], 0.5f * e.relg[x1]);
+        }
+        uint32_t t2;
+        if (TM == 0) {
+            t2 = tlo2;
+        } else if (TM == 1) {
+            const bool h0 = (uint32_t)e.tk32[c] - a1 >= span;
+            const bool h1 = (uint32_t)e.tk32[c + 1] - a1 >= span;
+            t2 = ((h0 ? thi2 : tlo2) & 0x0000FFFFu) | ((h1 ? thi2 : tlo2) & 0xFFFF0000u);
+        } else if (TM == 2) {
+            float v[2];
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const int32_t d = ht.t_rel - e.tk32[c + k];
+                uint32_t dt = (uint32_t)(d < 0 ? -d : d);
+                dt = min(dt, (uint32_t)INT32_MAX - 1u);
+                const float tv = e.tbh[lut_bucket(e.lut, dt)];
+                v[k] = ht.lane_const ? ht.tb_lo : tv;
+            }
+            t2 = pack_bf16x2(v[0], v[1]);
+        } else {
+            t2 = pack_bf16x2(e.tbh[bucket_search(e.thr, e.n_thr, abs_diff_u64(e.tsi, e.tk64[c]))],
+                             e.tbh[bucket_search(e.thr, e.n_thr,
+                                                 abs_diff_u64(e.tsi, e.tk64[c + 1]))]);
+        }
+        const uint32_t s2 = pack_bf16x2(__uint_as_float(s[2 * q]), __uint_as_float(s[2 * q + 1]));
+        const uint32_t h2 = add_bf16x2(fma_bf16x2(ha2, s2, r2), t2);
+        uint32_t a2 = fma_bf16x2(h2, tanh_bf16x2(h2), h2);
+        if (!FULL)
+            a2 &= (((vmask >> c) & 1u) ? 0x0000FFFFu : 0u) |
+                  (((vmask >> (c + 1)) & 1u) ? 0xFFFF0000u : 0u);
+        a[q] = a2;
+    }
+}
+
+// Inference: one 32-row x 32-key block (thread = row = TMEM lane), 8 keys per loop turn.
+// The loop is kept rolled: with a dozen of these bodies in the kernel, the instruction
+// cache, not load latency, limits the epilogue (unrolled or software-pipelined forms
+// measured 6-25 % slower on the long-history and windowed workloads).
+//   RD  the rel index rbase - c of every key lies within the guard-banded pair table:
+//       relp2[rbase - c] holds the biases of keys c and c + 1 (clamped entries in the
+//       guard bands), one shared load for two keys;
+//   otherwise each key's clamped index is read from the fp32 table.
+template <int TM, bool RD, bool FULL>
+__device__ __forceinline__ void fwd_quarter_inf(const FwdEpi &e, const HalfTime &ht,
+                                                uint32_t vmask)
+{
+    const uint32_t ha2 = pack_bf16x2(e.half_alpha, e.half_alpha);
+    const uint32_t tlo2 = pack_bf16x2(ht.tb_lo, ht.tb_lo);
+    const uint32_t thi2 = pack_bf16x2(ht.tb_hi, ht.tb_hi);
+    // one-boundary test as a single unsigned compare (see fwd_quarter)
+    const uint32_t a1 = (uint32_t)ht.cmpA + 1u;
+    const int64_t sp = (int64_t)ht.cmpB - (int64_t)ht.cmpA - 1;
+    const uint32_t span = sp > 0 ? (uint32_t)sp : 0u;
+    uint32_t s0[8], a[4];
+#pragma unroll 1
+    for (int ch = 0; ch < 4; ++ch) {
+        tmem_ld8(e.t_s + ch * 8, s0);
+        tmem_wait_ld();
+        reg_fence(s0);
+        inf_chunk<TM, RD, FULL>(e, ht, vmask, ch * 8, s0, ha2, tlo2, thi2, a1, span, a);
+        tmem_st4(e.t_a + ch * 4, a);
+    }
+}
+
 template <int DQK, int DV, bool SPLIT>
 __global__ void __launch_bounds__(kTcThreads, 1)
     fwd_tc_kernel(const __grid_constant__ FwdTcArgs args)
@@ -259,16 +355,26 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         *lut_valid = 1;
     }
     if (warp == 2) tmem_alloc(slot, kTmemCols);
-    // Tables hold half the bias.  The inference variant also scales by kTruncBump: its h is
-    // cut to bf16 by dropping the low 16 bits, and the bump removes the mean bias of that
-    // truncation (remaining error within one bf16 ulp).
-    const float tscale = SPLIT ? 0.5f : 0.5f * kTruncBump;
+    // Tables hold half the bias.  Training: the fp32 rel table.  Inference: bf16 key pairs,
+    // entry x = {rel[c(x)], rel[c(x-1)]} / 2 for x in [-kRelGuard, R - 1 + kRelGuard], with
+    // c() the clamp into [0, R-1] (zeros without a table).
+    const float tscale = 0.5f;
     for (int x = threadIdx.x; x < p.n_thr; x += kTcThreads) thr[x] = p.thr[x];
     for (int x = threadIdx.x; x < p.NB; x += kTcThreads) tbh[x] = tscale * p.tb[x];
-    const bool rel_in_smem = p.R <= kRelSmemMax;
-    if (rel_in_smem)
-        for (int x = threadIdx.x; x < p.R; x += kTcThreads) relh[x] = tscale * p.rel[x];
-    if (p.R == 0 && threadIdx.x == 0) relh[0] = 0.f;   // read, times zero bias, without a table
+    const bool rel_in_smem = SPLIT ? p.R <= kRelSmemMax : p.R <= kRelPairMax;
+    uint32_t *relp2 = reinterpret_cast<uint32_t *>(relh) + kRelGuard;
+    if (rel_in_smem) {
+        if (SPLIT) {
+            for (int x = threadIdx.x; x < p.R; x += kTcThreads) relh[x] = tscale * p.rel[x];
+        } else {
+            const int Re = p.R > 0 ? p.R : 1;
+            for (int x = threadIdx.x - kRelGuard; x < Re + kRelGuard; x += kTcThreads) {
+                const int x0 = min(max(x, 0), Re - 1), x1 = min(max(x - 1, 0), Re - 1);
+                relp2[x] = p.R > 0 ? pack_bf16x2(tscale * p.rel[x0], tscale * p.rel[x1]) : 0u;
+            }
+        }
+    }
+    if (p.R == 0 && threadIdx.x == 0 && SPLIT) relh[0] = 0.f;   // read, times zero bias
     fill_seq_tiles(p, kTcThreads);
     for (int b = blockIdx.x; b < p.B; b += gridDim.x) {   // rows no unit writes: zero Y
         RowRange rr[3];
@@ -507,7 +613,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const bool use_rel = p.R > 0;
         const float *relp = rel_in_smem ? relh : p.rel;
         const float rel_sc = rel_in_smem ? 1.0f : tscale;  // relp * rel_sc = scaled half rel bias
-        const float half_alpha = SPLIT ? 0.5f * p.alpha : 0.5f * kTruncBump * p.alpha;
+        const float half_alpha = 0.5f * p.alpha;
         const bool lut_ok = *lut_valid != 0;
         UnitFeed<FEED_WARP, false, BM> un(p, ring, args.nqt);
         int n = 0, g = 0;
@@ -535,9 +641,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 const int rbase = pi - jq;            // rel index of key jq + c is rbase - c
                 // a 32 x 32 block without a valid pair only writes zeros into A
                 const bool blk_any = __any_sync(0xffffffffu, vmask != 0u);
-                // without a rel table the clamped path reads the single zero entry
+                // training: without a rel table the clamped path reads the single zero entry;
+                // inference: the guard bands take indices up to kRelGuard outside the table
+                const int guard = SPLIT ? 0 : kRelGuard;
+                const int rb_ = use_rel ? rbase : 0;
                 const bool rdirect =
-                    use_rel && __all_sync(0xffffffffu, rbase - (QW - 1) >= 0 && rbase <= p.R - 1);
+                    (SPLIT ? use_rel : rel_in_smem) &&
+                    __all_sync(0xffffffffu, rb_ - (QW - 1) >= -guard &&
+                                                rb_ <= (use_rel ? p.R : 1) - 1 + guard);
                 HalfTime ht = {};
                 int tmode = 0;
                 if (use_ts) {
@@ -553,6 +664,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 e.tk64 = tsk + st * BN + wq * QW;
                 e.relp = use_rel ? relp : relh;
                 e.rel_sc = rel_sc;
+                e.relp2 = relp2;
+                e.relg = use_rel ? p.rel : relh;
                 e.rbase = use_rel ? rbase : 0;
                 e.R = use_rel ? p.R : 1;
                 e.half_alpha = half_alpha;
@@ -573,6 +686,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     // this quarter's A columns (SPLIT: hi and lo parts, 32 columns)
                     tmem_zero16(e.t_a);
                     if constexpr (SPLIT) tmem_zero16(e.t_a + 16);
+                } else if (!SPLIT) {
+                    if (tmode == 3) fwd_quarter_inf<3, false, false>(e, ht, vmask);
+                    else if (!rdirect) {
+                        if (tmode == 0) fwd_quarter_inf<0, false, false>(e, ht, vmask);
+                        else if (tmode == 1) fwd_quarter_inf<1, false, false>(e, ht, vmask);
+                        else fwd_quarter_inf<2, false, false>(e, ht, vmask);
+                    } else {
+                        // fully valid blocks run the masked bodies too (vmask all ones): fewer
+                        // bodies measured faster than a specialised one (instruction cache)
+                        if (tmode == 0) fwd_quarter_inf<0, true, false>(e, ht, vmask);
+                        else if (tmode == 1) fwd_quarter_inf<1, true, false>(e, ht, vmask);
+                        else fwd_quarter_inf<2, true, false>(e, ht, vmask);
+                    }
                 } else if (tmode == 3) {
                     fwd_quarter<3, false, false, SPLIT>(e, ht, vmask);
                 } else if (full && rdirect) {

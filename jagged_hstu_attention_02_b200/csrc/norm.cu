@@ -6,49 +6,13 @@
 // variance, eps inside the square root, no affine.  Other widths use the general kernels
 // in simt.cu.
 #include "kernels.h"
+#include "lnrow.cuh"
 
 namespace hstu {
 
 namespace {
 
 constexpr int kRows = 8;                  // tokens (warps) per 256-thread block
-
-template <typename T> struct Vec4;
-template <> struct Vec4<float> {
-    using type = float4;
-    static __device__ __forceinline__ void unpack(const float4 &v, float (&f)[4])
-    {
-        f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
-    }
-    static __device__ __forceinline__ float4 pack(const float (&f)[4])
-    {
-        return make_float4(f[0], f[1], f[2], f[3]);
-    }
-};
-template <> struct Vec4<__nv_bfloat16> {
-    using type = uint2;
-    static __device__ __forceinline__ void unpack(const uint2 &v, float (&f)[4])
-    {
-        f[0] = __uint_as_float(v.x << 16);
-        f[1] = __uint_as_float(v.x & 0xFFFF0000u);
-        f[2] = __uint_as_float(v.y << 16);
-        f[3] = __uint_as_float(v.y & 0xFFFF0000u);
-    }
-    static __device__ __forceinline__ uint2 pack(const float (&f)[4])
-    {
-        const __nv_bfloat162 a = __floats2bfloat162_rn(f[0], f[1]);
-        const __nv_bfloat162 b = __floats2bfloat162_rn(f[2], f[3]);
-        return make_uint2(*reinterpret_cast<const uint32_t *>(&a),
-                          *reinterpret_cast<const uint32_t *>(&b));
-    }
-};
-
-__device__ __forceinline__ float warp_sum(float v)
-{
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    return v;
-}
 
 // Forward: out = u * (y - mean) * rstd.  Lane l holds elements 128 c + 4 l .. +3.
 template <typename T, int NV>
@@ -67,32 +31,15 @@ __global__ void __launch_bounds__(32 * kRows)
     const typename V::type *ur = reinterpret_cast<const typename V::type *>(u + row * D) + lane;
     float v[NV][4];
     float uu[NV][4];
-    float sum = 0.f;
 #pragma unroll
     for (int c = 0; c < NV; ++c) {
         const float4 t = __ldg(yr + 32 * c);
         v[c][0] = t.x; v[c][1] = t.y; v[c][2] = t.z; v[c][3] = t.w;
         V::unpack(ur[32 * c], uu[c]);
-        sum += (t.x + t.y) + (t.z + t.w);
     }
-    const float mu = warp_sum(sum) * (1.0f / D);
-    float sq = 0.f;
-#pragma unroll
-    for (int c = 0; c < NV; ++c)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            v[c][e] -= mu;
-            sq = fmaf(v[c][e], v[c][e], sq);
-        }
-    const float rs = rsqrtf(warp_sum(sq) * (1.0f / D) + p.eps);
     typename V::type *orow = reinterpret_cast<typename V::type *>(out + row * D) + lane;
-#pragma unroll
-    for (int c = 0; c < NV; ++c) {
-        float o[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) o[e] = uu[c][e] * (v[c][e] * rs);
-        orow[32 * c] = V::pack(o);
-    }
+    float mu, rs;
+    ln_gate_regs<T, NV>(v, uu, p.eps, orow, &mu, &rs);
     if (lane == 0 && mean_out) {
         mean_out[row] = mu;
         rstd_out[row] = rs;
