@@ -39,7 +39,10 @@ def _capped_triangle(n: int, K) -> int:
     return K * (K + 1) // 2 + (n - K) * K
 
 
-def valid_pairs_seq(L: int, c: int = 0, t: int = 0, W: int = 0) -> int:
+CTX_SEES_HISTORY = 1   # mask variant: contextual rows see every key before the candidates
+
+
+def valid_pairs_seq(L: int, c: int = 0, t: int = 0, W: int = 0, flags: int = 0) -> int:
     """Number of valid (query, key) pairs of one sequence of length L."""
     if L <= 0:
         return 0
@@ -48,7 +51,8 @@ def valid_pairs_seq(L: int, c: int = 0, t: int = 0, W: int = 0) -> int:
         return L                       # only candidates: each sees itself
     K = (W + 1) if W > 0 else None
     hist = E - c
-    n = c * c                          # contextual rows see the contextual prefix
+    # contextual rows see the contextual prefix (or, variant, every key before the candidates)
+    n = c * (E if flags & CTX_SEES_HISTORY else c)
     n += c * hist                      # history rows see every contextual key ...
     n += _capped_triangle(hist, K)     # ... and causal (windowed) history keys
     seen = hist if K is None else min(hist, K)
@@ -61,7 +65,8 @@ def valid_pairs(batch) -> int:
     B = len(L)
     c = batch.num_contextuals if batch.num_contextuals is not None else np.zeros(B, np.int32)
     t = batch.num_targets if batch.num_targets is not None else np.zeros(B, np.int32)
-    return int(sum(valid_pairs_seq(int(L[b]), int(c[b]), int(t[b]), int(batch.max_attn_len))
+    f = int(getattr(batch, "mask_flags", 0))
+    return int(sum(valid_pairs_seq(int(L[b]), int(c[b]), int(t[b]), int(batch.max_attn_len), f)
                    for b in range(B)))
 
 
@@ -175,7 +180,8 @@ def bwd_attn_bytes(batch) -> int:
 
 # ------------------------------------------------------------------ visited tiles
 
-def tiles_with_pairs_seq(L: int, c: int = 0, t: int = 0, W: int = 0, tile: int = 128) -> int:
+def tiles_with_pairs_seq(L: int, c: int = 0, t: int = 0, W: int = 0, tile: int = 128,
+                         flags: int = 0) -> int:
     """(query tile, key tile) pairs of one sequence that hold at least one valid pair: the
     tiles a kernel that skips empty tiles must visit.  Per query tile, the union of its
     rows' valid key ranges: the contextual prefix (every row), the history rows' causal
@@ -195,6 +201,8 @@ def tiles_with_pairs_seq(L: int, c: int = 0, t: int = 0, W: int = 0, tile: int =
 
         if c > 0:
             add(0, c - 1)                                     # contextual keys / prefix rows
+            if flags & CTX_SEES_HISTORY and i0 < c:
+                add(0, E - 1)                                 # contextual rows: the history
         ra, rb = max(i0, c), min(i1, E - 1)                   # history rows
         if ra <= rb:
             add(max(c, ra - W) if W > 0 else c, rb)
@@ -212,5 +220,6 @@ def tiles_with_pairs(batch, tile: int = 128) -> int:
     B = len(L)
     c = batch.num_contextuals if batch.num_contextuals is not None else np.zeros(B, np.int32)
     t = batch.num_targets if batch.num_targets is not None else np.zeros(B, np.int32)
+    f = int(getattr(batch, "mask_flags", 0))
     return int(sum(tiles_with_pairs_seq(int(L[b]), int(c[b]), int(t[b]),
-                                        int(batch.max_attn_len), tile) for b in range(B)))
+                                        int(batch.max_attn_len), tile, f) for b in range(B)))

@@ -28,14 +28,16 @@ TOKEN_KEYS = ("q", "k", "v", "u", "timestamps", "dout")
 SEQ_KEYS = ("num_contextuals", "num_targets")
 
 
-def sequence_work(seq_offsets, num_contextuals=None, num_targets=None, max_attn_len=0):
+def sequence_work(seq_offsets, num_contextuals=None, num_targets=None, max_attn_len=0,
+                  mask_flags=0):
     """Valid (unmasked) pairs per sequence, per head."""
     offs = np.asarray(seq_offsets, dtype=np.int64)
     B = len(offs) - 1
     ctx = np.zeros(B, np.int64) if num_contextuals is None else np.asarray(num_contextuals)
     tgt = np.zeros(B, np.int64) if num_targets is None else np.asarray(num_targets)
     return np.array([accounting.valid_pairs_seq(int(offs[b + 1] - offs[b]), int(ctx[b]),
-                                                int(tgt[b]), int(max_attn_len))
+                                                int(tgt[b]), int(max_attn_len),
+                                                int(mask_flags))
                      for b in range(B)], dtype=np.int64)
 
 

@@ -51,6 +51,7 @@ class Batch:
     ln_eps: float = float(np.float32(1e-5))
     dout: Optional[np.ndarray] = None       # float32 [T, H*d_v] (backward workloads)
     name: str = ""
+    mask_flags: int = 0             # mask variants: 1 contextual rows see the history, 2 |rel|
 
     @property
     def batch(self) -> int:
@@ -96,7 +97,7 @@ def make_batch(rng: np.random.Generator, lengths: Sequence[int], num_heads: int,
                rel_bias_len: int = 0, time_bias_len: int = 0, time_gap_mean: float = 3600.0,
                ts_base: int = 1_600_000_000, alpha: Optional[float] = None,
                max_seqlen: Optional[int] = None, bias_std: float = 0.1,
-               with_dout: bool = False, name: str = "") -> Batch:
+               with_dout: bool = False, name: str = "", mask_flags: int = 0) -> Batch:
     """Draw one jagged batch.  Draw order: timestamps, q, k, v, u, rel table, time table, dout.
 
     `contextuals` / `targets` are an int (same for every sequence) or a per-sequence list.
@@ -145,7 +146,7 @@ def make_batch(rng: np.random.Generator, lengths: Sequence[int], num_heads: int,
     return Batch(num_heads=H, d_qk=d_qk, d_v=d_v, dtype=dtype, seq_offsets=offsets,
                  num_contextuals=ctx, num_targets=tgt, timestamps=ts, q=q, k=k, v=v, u=u,
                  rel_bias=rel, time_bias=tb, alpha=f32(alpha), max_attn_len=int(max_attn_len),
-                 max_seqlen=int(max_seqlen), dout=dout, name=name)
+                 max_seqlen=int(max_seqlen), dout=dout, name=name, mask_flags=int(mask_flags))
 
 
 # ------------------------------------------------------------------ the five workloads

@@ -20,8 +20,12 @@ def _silu(x):
     return x / (1.0 + np.exp(-x))
 
 
-def _mask_dense(L, c, t, W, N):
-    """[N, N] bool mask of one sequence padded to N (rows = queries)."""
+CTX_SEES_HISTORY, REL_ABS = 1, 2   # mask variants, as in the jagged oracle
+
+
+def _mask_dense(L, c, t, W, N, flags=0):
+    """[N, N] bool mask of one sequence padded to N (rows = queries).  With CTX_SEES_HISTORY
+    the contextual rows see every key before the candidates instead of the prefix only."""
     i = np.arange(N)[:, None]
     j = np.arange(N)[None, :]
     E = L - t
@@ -32,7 +36,8 @@ def _mask_dense(L, c, t, W, N):
     ctx_key = j < c
     window_ok = (pi - j <= W) if W > 0 else np.ones_like(cand_key)
     hist = (j <= pi) & window_ok
-    valid = np.where(cand_key, i == j, np.where(ctx_row, ctx_key, ctx_key | hist))
+    ctx_row_keys = (j < E) if flags & CTX_SEES_HISTORY else ctx_key
+    valid = np.where(cand_key, i == j, np.where(ctx_row, ctx_row_keys, ctx_key | hist))
     return valid & in_seq
 
 
@@ -59,8 +64,10 @@ def fwd(b):
         p = np.where(pos < E, pos, E - 1) if E > 0 else pos
         p = np.clip(p, 0, max(L - 1, 0))
         bias = np.zeros((N, N))
+        flags = int(getattr(b, "mask_flags", 0))
         if b.rel_bias_len > 0:
-            r = np.clip(p[:, None] - p[None, :], 0, b.rel_bias_len - 1)
+            d = p[:, None] - p[None, :]
+            r = np.clip(np.abs(d) if flags & REL_ABS else d, 0, b.rel_bias_len - 1)
             bias += np.asarray(b.rel_bias, np.float64)[r]
         if b.time_bias_len > 0 and L > 0:
             ts = np.zeros(N, dtype=np.int64)
@@ -69,7 +76,7 @@ def fwd(b):
             bk = np.floor(np.log(dt + 1.0) / b.time_bucket_div)
             bk = np.clip(bk, 0, b.time_bias_len - 1).astype(np.int64)
             bias += np.asarray(b.time_bias, np.float64)[bk]
-        m = _mask_dense(L, c, t, int(b.max_attn_len), N)
+        m = _mask_dense(L, c, t, int(b.max_attn_len), N, flags)
         for h in range(H):
             scores = b.alpha * (q[s, :, h] @ k[s, :, h].T) + bias
             a = _silu(scores) / N

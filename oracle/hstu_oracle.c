@@ -45,6 +45,12 @@
  *  - alpha multiplies q.k only, not the bias;
  *  - one rel table and one time table shared by all heads.
  *
+ * Two variants of the mask family, as flags (both off by default):
+ *  - ORACLE_CTX_SEES_HISTORY: contextual rows attend to every key before the candidates
+ *    (the contextual prefix and the whole history), not only to the contextual prefix;
+ *  - ORACLE_REL_ABS: the rel index is min(|p(i) - p(j)|, R-1) rather than clamp(p(i) - p(j),
+ *    0, R-1), so bidirectional pairs with p(i) < p(j) index by their distance.
+ *
  * All inputs are fp64 copies of the values the device sees (bf16 inputs are rounded
  * by the input generator and upcast exactly).  Layouts: q,k [T,H,dqk], v [T,H,dv],
  * u, out, y [T,H*dv], row-major; column index of (head h, element e) is h*dv+e.
@@ -82,6 +88,9 @@ int64_t hstu_oracle_time_bucket(int64_t dt, double div, int64_t NB)
     return (int64_t)f;
 }
 
+#define ORACLE_CTX_SEES_HISTORY 1
+#define ORACLE_REL_ABS 2
+
 static int64_t clamped_pos(int64_t x, int64_t E)
 {
     if (E <= 0) return x;
@@ -89,11 +98,12 @@ static int64_t clamped_pos(int64_t x, int64_t E)
 }
 
 /* The mask predicate of the reading above, for local positions i (query) and j (key). */
-static int oracle_valid(int64_t i, int64_t j, int64_t L, int64_t c, int64_t t, int64_t W)
+static int oracle_valid(int64_t i, int64_t j, int64_t L, int64_t c, int64_t t, int64_t W,
+                        int64_t flags)
 {
     int64_t E = L - t;
     if (j >= E) return i == j;
-    if (i < c) return j < c;
+    if (i < c) return (flags & ORACLE_CTX_SEES_HISTORY) ? 1 : j < c;
     if (j < c) return 1;
     int64_t pi = clamped_pos(i, E);
     if (j > pi) return 0;
@@ -102,28 +112,34 @@ static int oracle_valid(int64_t i, int64_t j, int64_t L, int64_t c, int64_t t, i
 }
 
 /* Mask of one sequence as an L*L byte matrix (row i = query).  Returns the valid-pair count. */
-int64_t hstu_oracle_mask(int64_t L, int64_t c, int64_t t, int64_t W, uint8_t *mask)
+int64_t hstu_oracle_mask_flags(int64_t L, int64_t c, int64_t t, int64_t W, int64_t flags,
+                               uint8_t *mask)
 {
     int64_t n = 0;
     for (int64_t i = 0; i < L; ++i)
         for (int64_t j = 0; j < L; ++j) {
-            int v = oracle_valid(i, j, L, c, t, W);
+            int v = oracle_valid(i, j, L, c, t, W, flags);
             if (mask) mask[i * L + j] = (uint8_t)v;
             n += v;
         }
     return n;
 }
 
+int64_t hstu_oracle_mask(int64_t L, int64_t c, int64_t t, int64_t W, uint8_t *mask)
+{
+    return hstu_oracle_mask_flags(L, c, t, W, 0, mask);
+}
+
 /* Rows [r0, r0+nrows) x keys [0, ncols) of the same mask, positions past the sequence's end
  * (>= L) counted invalid; row r - r0 of `mask` has ncols bytes.  Returns the valid count. */
-int64_t hstu_oracle_mask_rows(int64_t L, int64_t c, int64_t t, int64_t W, int64_t r0,
-                              int64_t nrows, int64_t ncols, uint8_t *mask)
+int64_t hstu_oracle_mask_rows(int64_t L, int64_t c, int64_t t, int64_t W, int64_t flags,
+                              int64_t r0, int64_t nrows, int64_t ncols, uint8_t *mask)
 {
     int64_t n = 0;
     for (int64_t r = 0; r < nrows; ++r)
         for (int64_t j = 0; j < ncols; ++j) {
             int64_t i = r0 + r;
-            int v = i < L && j < L && oracle_valid(i, j, L, c, t, W);
+            int v = i < L && j < L && oracle_valid(i, j, L, c, t, W, flags);
             mask[r * ncols + j] = (uint8_t)v;
             n += v;
         }
@@ -141,6 +157,7 @@ typedef struct {
     int64_t NB;
     double div, alpha;
     int64_t W, N;
+    int64_t flags;
 } oracle_problem;
 
 /* Bias b_ij for local positions i, j of a sequence starting at global row s0. */
@@ -153,7 +170,7 @@ static double oracle_bias(const oracle_problem *P, int64_t s0, int64_t E, int64_
     *bucket = -1;
     if (P->R > 0) {
         int64_t r = pi - pj;
-        if (r < 0) r = 0;
+        if (r < 0) r = (P->flags & ORACLE_REL_ABS) ? -r : 0;
         if (r > P->R - 1) r = P->R - 1;
         *rel_idx = r;
         b += P->rel[r];
@@ -184,11 +201,11 @@ int hstu_oracle_fwd(int64_t B, int64_t H, int64_t dqk, int64_t dv, const int64_t
                     const int32_t *ctx, const int32_t *tgt, const int64_t *ts, const double *q,
                     const double *k, const double *v, const double *u, const double *rel,
                     int64_t R, const double *tb, int64_t NB, double div, double alpha,
-                    int64_t max_attn_len, int64_t N, double eps, double *out, double *y,
-                    double *mean, double *rstd)
+                    int64_t max_attn_len, int64_t N, double eps, int64_t flags, double *out,
+                    double *y, double *mean, double *rstd)
 {
     oracle_problem P = {B, H, dqk, dv, offsets, ctx, tgt, ts, rel, R, tb, NB, div, alpha,
-                        max_attn_len, N};
+                        max_attn_len, N, flags};
     const int64_t D = H * dv;
     int bad = 0;
     for (int64_t b = 0; b < B; ++b) {
@@ -208,7 +225,7 @@ int hstu_oracle_fwd(int64_t B, int64_t H, int64_t dqk, int64_t dv, const int64_t
             for (int64_t h = 0; h < H; ++h) {
                 const double *qi = q + ((s0 + i) * H + h) * dqk;
                 for (int64_t j = 0; j < L; ++j) {
-                    if (!oracle_valid(i, j, L, c, t, max_attn_len)) continue;
+                    if (!oracle_valid(i, j, L, c, t, max_attn_len, flags)) continue;
                     const double *kj = k + ((s0 + j) * H + h) * dqk;
                     double dot = 0.0;
                     for (int64_t e = 0; e < dqk; ++e) dot += qi[e] * kj[e];
@@ -252,11 +269,12 @@ int hstu_oracle_bwd(int64_t B, int64_t H, int64_t dqk, int64_t dv, const int64_t
                     const int32_t *ctx, const int32_t *tgt, const int64_t *ts, const double *q,
                     const double *k, const double *v, const double *u, const double *rel,
                     int64_t R, const double *tb, int64_t NB, double div, double alpha,
-                    int64_t max_attn_len, int64_t N, double eps, const double *dout, double *dq,
-                    double *dk, double *dvv, double *du, double *drel, double *dtb)
+                    int64_t max_attn_len, int64_t N, double eps, int64_t flags,
+                    const double *dout, double *dq, double *dk, double *dvv, double *du,
+                    double *drel, double *dtb)
 {
     oracle_problem P = {B, H, dqk, dv, offsets, ctx, tgt, ts, rel, R, tb, NB, div, alpha,
-                        max_attn_len, N};
+                        max_attn_len, N, flags};
     const int64_t D = H * dv;
     int64_t T = offsets[B];
     int bad = 0;
@@ -272,7 +290,7 @@ int hstu_oracle_bwd(int64_t B, int64_t H, int64_t dqk, int64_t dv, const int64_t
     double *rstd = (double *)malloc(sizeof(double) * (size_t)(T + 1));
     double *dy = (double *)malloc(sizeof(double) * (size_t)(T * D + 1));
     hstu_oracle_fwd(B, H, dqk, dv, offsets, ctx, tgt, ts, q, k, v, u, rel, R, tb, NB, div, alpha,
-                    max_attn_len, N, eps, NULL, y, mean, rstd);
+                    max_attn_len, N, eps, flags, NULL, y, mean, rstd);
 
     /* O = U (.) Zhat, Zhat = (Y - mu) * rstd.  dU = dO (.) Zhat; dZhat = dO (.) U;
      * dY = rstd * (dZhat - mean(dZhat) - Zhat * mean(dZhat (.) Zhat)). */
@@ -314,7 +332,7 @@ int hstu_oracle_bwd(int64_t B, int64_t H, int64_t dqk, int64_t dv, const int64_t
                     const double *qi = q + ((s0 + i) * H + h) * dqk;
                     const double *dyi = dy + (s0 + i) * D + h * dv;
                     for (int64_t j = 0; j < L; ++j) {
-                        if (!oracle_valid(i, j, L, c, t, max_attn_len)) continue;
+                        if (!oracle_valid(i, j, L, c, t, max_attn_len, flags)) continue;
                         const double *kj = k + ((s0 + j) * H + h) * dqk;
                         const double *vj = v + ((s0 + j) * H + h) * dv;
                         double dot = 0.0;

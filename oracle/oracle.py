@@ -35,10 +35,12 @@ def lib():
         L.hstu_oracle_time_bucket.argtypes = [_I64, _F64, _I64]
         L.hstu_oracle_mask.restype = _I64
         L.hstu_oracle_mask.argtypes = [_I64, _I64, _I64, _I64, _P_U8]
+        L.hstu_oracle_mask_flags.restype = _I64
+        L.hstu_oracle_mask_flags.argtypes = [_I64] * 5 + [_P_U8]
         common = [_I64, _I64, _I64, _I64, _P_I64, _P_I32, _P_I32, _P_I64, _P_F64, _P_F64,
-                  _P_F64, _P_F64, _P_F64, _I64, _P_F64, _I64, _F64, _F64, _I64, _I64, _F64]
+                  _P_F64, _P_F64, _P_F64, _I64, _P_F64, _I64, _F64, _F64, _I64, _I64, _F64, _I64]
         L.hstu_oracle_mask_rows.restype = _I64
-        L.hstu_oracle_mask_rows.argtypes = [_I64] * 7 + [_P_U8]
+        L.hstu_oracle_mask_rows.argtypes = [_I64] * 8 + [_P_U8]
         L.hstu_oracle_fwd.restype = ctypes.c_int
         L.hstu_oracle_fwd.argtypes = common + [_P_F64] * 4
         L.hstu_oracle_bwd.restype = ctypes.c_int
@@ -63,18 +65,25 @@ def time_bucket(dt: int, div: float = 0.301, nb: int = 128) -> int:
     return int(lib().hstu_oracle_time_bucket(int(dt), float(div), int(nb)))
 
 
-def mask(L: int, c: int = 0, t: int = 0, W: int = 0):
+# mask variants (flags): contextual rows see the whole history; rel index |p(i) - p(j)|
+CTX_SEES_HISTORY, REL_ABS = 1, 2
+
+
+def mask(L: int, c: int = 0, t: int = 0, W: int = 0, flags: int = 0):
     """(L x L uint8 mask, valid-pair count) of one sequence; row = query position."""
     m = np.zeros((max(L, 1), max(L, 1)), dtype=np.uint8)[:L, :L].copy()
-    n = lib().hstu_oracle_mask(L, c, t, W, _ptr(m, ctypes.c_uint8))
+    if flags:
+        n = lib().hstu_oracle_mask_flags(L, c, t, W, flags, _ptr(m, ctypes.c_uint8))
+    else:
+        n = lib().hstu_oracle_mask(L, c, t, W, _ptr(m, ctypes.c_uint8))
     return m, int(n)
 
 
-def mask_rows(L: int, c: int, t: int, W: int, r0: int, nrows: int, ncols: int):
+def mask_rows(L: int, c: int, t: int, W: int, r0: int, nrows: int, ncols: int, flags: int = 0):
     """Rows [r0, r0+nrows) x keys [0, ncols) of the mask of one sequence (positions >= L
     invalid), as a uint8 matrix."""
     m = np.zeros((nrows, ncols), dtype=np.uint8)
-    lib().hstu_oracle_mask_rows(L, c, t, W, r0, nrows, ncols, _ptr(m, ctypes.c_uint8))
+    lib().hstu_oracle_mask_rows(L, c, t, W, flags, r0, nrows, ncols, _ptr(m, ctypes.c_uint8))
     return m
 
 
@@ -95,7 +104,8 @@ def _common_args(b, keep):
             _ptr(q, ctypes.c_double), _ptr(k, ctypes.c_double), _ptr(v, ctypes.c_double),
             _ptr(u, ctypes.c_double), _ptr(rel, ctypes.c_double), b.rel_bias_len,
             _ptr(tb, ctypes.c_double), b.time_bias_len, float(b.time_bucket_div),
-            float(b.alpha), int(b.max_attn_len), int(b.max_seqlen), float(b.ln_eps)]
+            float(b.alpha), int(b.max_attn_len), int(b.max_seqlen), float(b.ln_eps),
+            int(getattr(b, "mask_flags", 0))]
 
 
 def fwd(b):

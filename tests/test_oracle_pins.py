@@ -416,3 +416,80 @@ def test_visited_tile_count_is_the_tiles_holding_a_valid_pair(L, c, t, W):
     brute = sum(1 for a in range(nt) for b in range(nt)
                 if m[a * 128:(a + 1) * 128, b * 128:(b + 1) * 128].any())
     assert accounting.tiles_with_pairs_seq(L, c, t, W) == brute
+
+
+# ---------------------------------------------------------------- mask variants (flags)
+
+def test_mask_variant_hand_examples(golden_dir):
+    """The two variants of the mask family against hand-derived masks; the dense
+    formulation and the closed-form count agree."""
+    lines = [ln.split("#")[0].strip() for ln in open(f"{golden_dir}/mask_examples_variants.txt")]
+    lines = [ln for ln in lines if ln]
+    i = 0
+    while i < len(lines):
+        _, L, c, t, W, f, n = lines[i].split()
+        L, c, t, W, f, n = int(L), int(c), int(t), int(W), int(f), int(n)
+        m = np.array([[int(ch) for ch in row] for row in lines[i + 1:i + 1 + L]], np.uint8)
+        got, cnt = oracle.mask(L, c, t, W, f)
+        assert np.array_equal(got, m), (L, c, t, W, f)
+        assert cnt == n == int(m.sum())
+        assert accounting.valid_pairs_seq(L, c, t, W, f) == n
+        assert np.array_equal(dense._mask_dense(L, c, t, W, L, f).astype(np.uint8), m)
+        i += 1 + L
+
+
+@pytest.mark.parametrize("W", [0, 2, 7])
+def test_mask_variant_counts_and_structure(W):
+    """Contextual rows see every key before the candidates and nothing after; every other
+    row keeps the default mask; counts follow the closed form."""
+    for L in [1, 2, 9, 23]:
+        for c in range(0, min(L, 4) + 1):
+            for t in range(0, L - c + 1, max(1, (L - c) // 3 or 1)):
+                base, _ = oracle.mask(L, c, t, W)
+                m, cnt = oracle.mask(L, c, t, W, oracle.CTX_SEES_HISTORY)
+                E = L - t
+                assert m[:c, :E].all() and not m[:c, E:].any()
+                assert np.array_equal(m[c:], base[c:])
+                assert cnt == accounting.valid_pairs_seq(L, c, t, W, 1)
+                assert np.array_equal(oracle.mask(L, c, t, W, oracle.REL_ABS)[0], base)
+
+
+def test_rel_abs_indexes_bidirectional_pairs_by_distance():
+    """Q = K = 0, one-hot rel table at r: contextual rows see later keys at p(j) - p(i) > 0.
+    Default: that index clamps to 0.  With the |p(i) - p(j)| variant it is the distance."""
+    silu1 = 1.0 / (1.0 + 1.0 / E_CONST)
+    for flags in (oracle.REL_ABS, oracle.REL_ABS | oracle.CTX_SEES_HISTORY):
+        for r in (1, 2):
+            b = _empty_batch([6], 1, 16, 4, ctx=3, R=4)
+            b.mask_flags = flags
+            b.rel_bias[r] = 1.0
+            b.v[:, 0, :] = np.random.default_rng(r).standard_normal((6, 4))
+            y = oracle.fwd(b)["y"] * b.max_seqlen
+            V = b.v[:, 0, :].astype(np.float64)
+            see = 6 if flags & oracle.CTX_SEES_HISTORY else 3   # keys of the contextual rows
+            for i in range(3):
+                expect = sum(V[j] for j in range(see) if abs(i - j) == r)
+                assert np.allclose(y[i], silu1 * expect if np.ndim(expect) else 0 * V[0],
+                                   atol=1e-14), (flags, r, i)
+            for i in range(3, 6):   # history rows: causal, the distance is i - j >= 0
+                expect = sum(V[j] for j in range(0, i + 1) if i - j == r)
+                assert np.allclose(y[i], silu1 * expect, atol=1e-14), (flags, r, i)
+
+
+@pytest.mark.parametrize("flags", [1, 2, 3])
+def test_mask_variants_jagged_equals_dense(flags):
+    b = synth.make_batch(np.random.default_rng(60 + flags), [9, 30, 1, 14], 2, 8, 8, "f32",
+                         contextuals=[2, 4, 0, 3], targets=[3, 5, 1, 0], max_attn_len=5,
+                         rel_bias_len=12, time_bias_len=32, mask_flags=flags)
+    a, d = oracle.fwd(b), dense.fwd(b)
+    for key in ("out", "y", "mean", "rstd"):
+        assert np.allclose(a[key], d[key], rtol=1e-12, atol=1e-12), key
+
+
+@pytest.mark.parametrize("flags", [1, 2, 3])
+def test_mask_variants_backward_finite_differences(flags):
+    b = synth.make_batch(np.random.default_rng(70 + flags), [9, 17, 3], 2, 8, 8, "f32",
+                         contextuals=[2, 3, 0], targets=[3, 2, 1], max_attn_len=4,
+                         rel_bias_len=12, time_bias_len=32, mask_flags=flags)
+    dout = np.random.default_rng(80 + flags).standard_normal(b.u.shape)
+    _fd_check(b, dout, samples=8)
