@@ -32,6 +32,10 @@
  *                  i < c  : j < c                       (contextual rows: bidirectional prefix)
  *                  j < c  : true                        (contextual keys: seen by every row)
  *                  else   : j <= p(i) && (W <= 0 || p(i) - j <= W)
+ * Two variants, selected by params->flags: HSTU_FLAG_CTX_SEES_HISTORY makes a contextual row
+ * see every key before the candidates (i < c : j < E); HSTU_FLAG_REL_ABS indexes the rel
+ * table by min(|p(i) - p(j)|, R-1) instead of clamp(p(i) - p(j), 0, R-1), so bidirectional
+ * pairs with p(i) < p(j) use their distance.
  *
  * Layouts (all row-major, packed over the T = seq_offsets[B] tokens of the batch):
  *    q, k        [T, H, d_qk]        dtype            dq, dk   [T, H, d_qk]  dtype
@@ -85,6 +89,10 @@ typedef enum {
 
 typedef enum { HSTU_F32 = 0, HSTU_BF16 = 1 } hstu_dtype_t;
 
+/* Mask variants (params->flags). */
+#define HSTU_FLAG_CTX_SEES_HISTORY 0x1   /* contextual rows attend to every non-candidate key */
+#define HSTU_FLAG_REL_ABS          0x2   /* rel index min(|p(i) - p(j)|, R - 1) */
+
 /* Bits of the device status word. */
 #define HSTU_DEV_BAD_OFFSETS   0x1   /* seq_offsets not non-decreasing / not ending at T */
 #define HSTU_DEV_BAD_COUNTS    0x2   /* num_contextuals/num_targets negative or c + t > L */
@@ -105,7 +113,7 @@ typedef struct {
     int32_t time_bias_len;    /* NB in 0..256; 0 = no time bias (timestamps may be NULL) */
     double time_bucket_div;   /* > 0, e.g. 0.301 (natural log) */
     int32_t dtype;            /* hstu_dtype_t of q,k,v,u,out,dout,dq,dk,dv,du */
-    int32_t reserved;         /* must be 0 */
+    int32_t flags;            /* HSTU_FLAG_* mask variants (0: the default mask); other bits 0 */
 } hstu_attn_params_t;
 
 /* Workspace bytes hstu_attn_fwd needs for these params (saved_y NULL or not). */

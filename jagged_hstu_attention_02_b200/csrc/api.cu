@@ -65,7 +65,7 @@ const ThrEntry &thresholds(double div, int nb)
 hstu_status_t validate(const hstu_attn_params_t *p)
 {
     if (!p) return HSTU_ERR_INVALID_ARGUMENT;
-    if (p->reserved != 0) return HSTU_ERR_INVALID_ARGUMENT;
+    if (p->flags & ~(HSTU_FLAG_CTX_SEES_HISTORY | HSTU_FLAG_REL_ABS)) return HSTU_ERR_INVALID_ARGUMENT;
     if (p->batch < 0 || p->num_heads < 1 || p->total_tokens < 0) return HSTU_ERR_INVALID_ARGUMENT;
     if (p->max_seqlen < 1) return HSTU_ERR_INVALID_ARGUMENT;
     if (p->d_qk < 1 || p->d_v < 1 || p->d_qk > 256 || p->d_v > 256)
@@ -113,6 +113,7 @@ DevParams make_dev_params(const hstu_attn_params_t *p, const int64_t *offsets, c
     d.rel = rel;
     d.tb = tb;
     d.status = reinterpret_cast<int32_t *>(workspace);
+    d.flags = p->flags;
     d.wait_limit = g_wait_limit;
     d.stall_test = g_stall_test;
     if (d.NB > 0) {

@@ -57,8 +57,8 @@ __device__ __forceinline__ uint64_t range_bits(int a, int b, int jh)
 __device__ __forceinline__ uint64_t row_valid_bits(int i, int jh, const SeqInfo &s, int W)
 {
     if (i >= s.L) return 0ull;
+    if (i < s.c) return range_bits(0, (s.cfull ? s.E : s.c) - 1, jh);   // contextual row
     uint64_t m = range_bits(0, s.c - 1, jh);
-    if (i < s.c) return m;
     const int pi = clamp_pos(i, s.E);
     const int lo = W > 0 ? max(s.c, pi - W) : s.c;
     m |= range_bits(lo, min(pi, s.E - 1), jh);
@@ -112,6 +112,7 @@ __device__ __forceinline__ uint64_t col_valid_bits(int j, int ih, const SeqInfo 
     // every candidate row
     const int hi = W > 0 ? min(s.E - 1, j + W) : s.E - 1;
     uint64_t m = range_bits(max(j, s.c), hi, ih);
+    if (s.cfull) m |= range_bits(0, s.c - 1, ih);               // variant: contextual rows
     if (W <= 0 || (s.E - 1) - j <= W) m |= range_bits(s.E, s.L - 1, ih);
     return m;
 }

@@ -262,8 +262,7 @@ __device__ __forceinline__ void epi_block(const DevParams &p, const EpiBlock &e,
             } else if (KIND == 1) {
                 ri = cc >= e.fc ? e.rc : e.rbase + cc;
             } else {
-                const int rraw = min(i, e.Em1) - k.pj;
-                ri = rraw < 0 ? 0 : (rraw > p.R - 1 ? p.R - 1 : rraw);
+                ri = rel_index(min(i, e.Em1) - k.pj, p.R, (p.flags & HSTU_FLAG_REL_ABS) != 0);
             }
             bias[c] += e.relp[ri];
             bkv[c] = bk;

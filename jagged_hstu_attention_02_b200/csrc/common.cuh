@@ -31,6 +31,7 @@ struct DevParams {
     const int64_t *ts;
     const float *rel, *tb;
     int32_t *status;
+    int32_t flags;          // HSTU_FLAG_* mask variants
     long long wait_limit;   // cycles a pipeline wait may take before the kernel gives up
     int32_t stall_test;     // test only: the MMA issuer first waits on a barrier nothing completes
     // smallest |dt| of bucket k+1 (fp64-decided on the host), ascending
@@ -41,6 +42,7 @@ struct SeqInfo {
     int64_t start;
     int L, c, t, E;
     bool ok;
+    bool cfull;   // contextual rows see every key before the candidates (mask variant)
 };
 
 __device__ __forceinline__ void flag_error(const DevParams &p, int bits)
@@ -58,6 +60,7 @@ __device__ __forceinline__ SeqInfo load_seq(const DevParams &p, int b, bool repo
     s.c = p.ctx ? p.ctx[b] : 0;
     s.t = p.tgt ? p.tgt[b] : 0;
     s.ok = true;
+    s.cfull = (p.flags & HSTU_FLAG_CTX_SEES_HISTORY) != 0;
     int bits = 0;
     if (a < 0 || L < 0 || e > p.T) { bits |= HSTU_DEV_BAD_OFFSETS; }
     // the offsets must start at row 0 and end at row T
@@ -171,10 +174,18 @@ __device__ __forceinline__ void transpose_chunks(float4 (&x)[NCH])
 // p(x): candidates take the last history position.
 __device__ __forceinline__ int clamp_pos(int x, int E) { return (E > 0 && x >= E) ? E - 1 : x; }
 
+// Index into the rel table of positions with p(i) - p(j) = d: clamp(d, 0, R-1), or, with the
+// |p(i) - p(j)| variant, min(|d|, R-1).
+__device__ __forceinline__ int rel_index(int d, int R, bool rabs)
+{
+    if (d < 0) d = rabs ? -d : 0;
+    return d > R - 1 ? R - 1 : d;
+}
+
 __device__ __forceinline__ bool pair_valid(int i, int j, const SeqInfo &s, int W)
 {
     if (j >= s.E) return i == j;          // candidate key: itself only
-    if (i < s.c) return j < s.c;          // contextual row: bidirectional prefix
+    if (i < s.c) return s.cfull || j < s.c;   // contextual row: prefix (variant: all history)
     if (j < s.c) return true;             // contextual key: every row
     int pi = clamp_pos(i, s.E);
     return j <= pi && (W <= 0 || pi - j <= W);
@@ -189,6 +200,7 @@ __device__ __forceinline__ bool tile_any_valid(int i0, int i1, int j0, int j1, c
     j1 = min(j1, s.L - 1);
     if (i0 > i1 || j0 > j1) return false;
     if (j0 < s.c) return true;                              // contextual keys: every row
+    if (s.cfull && i0 < s.c && j0 < s.E) return true;       // variant: contextual rows see all
     int a = max(j0, s.E);
     if (a <= j1 && max(i0, a) <= min(i1, j1)) return true;  // candidate diagonal
     int ha = max(j0, s.c), hb = min(j1, s.E - 1);           // history keys

@@ -130,6 +130,8 @@ struct FwdEpi {
     const uint32_t *relp2;     // inference: bf16 pair table, relp2[x] = {rel[x], rel[x-1]} / 2
     const float *relg;         // inference, clamped blocks: the fp32 table (R >= 1 entries)
     int rbase, R;              // rel index of key c: rbase - c (clamped unless RD)
+    int cand0, rcand;          // clamped blocks: keys c >= cand0 are candidates, p(i) - p(j) = rcand
+    bool rabs;                 // rel index min(|p(i) - p(j)|, R-1) (mask variant)
     float half_alpha, alpha;
     const float *tbh;          // half time-bias table
     const LutEntry *lut;
@@ -171,7 +173,7 @@ __device__ __forceinline__ void fwd_quarter(const FwdEpi &e, const HalfTime &ht,
                 tb[c] = e.tbh[bucket_search(e.thr, e.n_thr, abs_diff_u64(e.tsi, e.tk64[cb + c]))];
             }
             int ri = e.rbase - cb - c;
-            if (!RD) ri = ri < 0 ? 0 : (ri > e.R - 1 ? e.R - 1 : ri);
+            if (!RD) ri = rel_index(cb + c < e.cand0 ? ri : e.rcand, e.R, e.rabs);
             rv[c] = e.relp[ri];
         }
         float2 bh[2];
@@ -246,9 +248,9 @@ __device__ __forceinline__ void inf_chunk(const FwdEpi &e, const HalfTime &ht, u
         if (RD) {
             r2 = e.relp2[e.rbase - c];           // guard-banded: no clamp needed here
         } else {
-            int x0 = e.rbase - c, x1 = x0 - 1;
-            x0 = x0 < 0 ? 0 : (x0 > e.R - 1 ? e.R - 1 : x0);
-            x1 = x1 < 0 ? 0 : (x1 > e.R - 1 ? e.R - 1 : x1);
+            // the key's own position p(j): candidate keys take the last history position
+            const int x0 = rel_index(c < e.cand0 ? e.rbase - c : e.rcand, e.R, e.rabs);
+            const int x1 = rel_index(c + 1 < e.cand0 ? e.rbase - c - 1 : e.rcand, e.R, e.rabs);
             r2 = pack_bf16x2(0.5f * e.relg[x0], 0.5f * e.relg[x1]);
         }
         uint32_t t2;
@@ -368,8 +370,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             for (int x = threadIdx.x; x < p.R; x += kTcThreads) relh[x] = tscale * p.rel[x];
         } else {
             const int Re = p.R > 0 ? p.R : 1;
+            const bool rabs = (p.flags & HSTU_FLAG_REL_ABS) != 0;
             for (int x = threadIdx.x - kRelGuard; x < Re + kRelGuard; x += kTcThreads) {
-                const int x0 = min(max(x, 0), Re - 1), x1 = min(max(x - 1, 0), Re - 1);
+                const int x0 = rel_index(x, Re, rabs), x1 = rel_index(x - 1, Re, rabs);
                 relp2[x] = p.R > 0 ? pack_bf16x2(tscale * p.rel[x0], tscale * p.rel[x1]) : 0u;
             }
         }
@@ -645,8 +648,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 // inference: the guard bands take indices up to kRelGuard outside the table
                 const int guard = SPLIT ? 0 : kRelGuard;
                 const int rb_ = use_rel ? rbase : 0;
+                // (the direct index uses j for p(j): right for candidate keys only when negative
+                // distances clamp to 0, so the |p(i) - p(j)| variant takes such blocks clamped)
+                const bool rabs = (p.flags & HSTU_FLAG_REL_ABS) != 0;
                 const bool rdirect =
-                    (SPLIT ? use_rel : rel_in_smem) &&
+                    (SPLIT ? use_rel : rel_in_smem) && (!rabs || jq + QW - 1 < s.E) &&
                     __all_sync(0xffffffffu, rb_ - (QW - 1) >= -guard &&
                                                 rb_ <= (use_rel ? p.R : 1) - 1 + guard);
                 HalfTime ht = {};
@@ -668,6 +674,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 e.relg = use_rel ? p.rel : relh;
                 e.rbase = use_rel ? rbase : 0;
                 e.R = use_rel ? p.R : 1;
+                e.cand0 = s.E > 0 ? s.E - jq : (1 << 30);   // E = 0: positions unclamped
+                e.rcand = use_rel ? pi - (s.E - 1) : 0;
+                e.rabs = rabs;
                 e.half_alpha = half_alpha;
                 e.alpha = p.alpha;
                 e.tbh = tbh;

@@ -43,7 +43,7 @@ __device__ __forceinline__ float pair_bias(const DevParams &p, const SmemHeader 
     *bk = -1;
     if (p.R > 0) {
         int r = pi - pj;
-        r = r < 0 ? 0 : (r > p.R - 1 ? p.R - 1 : r);
+        r = rel_index(r, p.R, (p.flags & HSTU_FLAG_REL_ABS) != 0);
         *ri = r;
         b += __ldg(p.rel + r);
     }

@@ -27,9 +27,13 @@ constexpr int kBlk = 32;     // the 32-wide blocks inside a tile the epilogues d
 struct TileIter {
     const SeqInfo &s;
     int i0, W, kt;
+    // (with the variant in which contextual rows see the whole history, a tile holding
+    // contextual rows starts from the last tile)
     __device__ TileIter(const SeqInfo &s_, int i0_, int W_)
         : s(s_), i0(i0_), W(W_),
-          kt(min((s_.L + kTile - 1) / kTile, max(i0_ / kTile, (s_.c - 1) / kTile) + 1)) {}
+          kt((s_.cfull && i0_ < s_.c)
+                 ? (s_.L + kTile - 1) / kTile
+                 : min((s_.L + kTile - 1) / kTile, max(i0_ / kTile, (s_.c - 1) / kTile) + 1)) {}
     __device__ bool next()
     {
         while (--kt >= 0)

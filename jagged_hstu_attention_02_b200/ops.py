@@ -42,7 +42,10 @@ class Params(ctypes.Structure):
                 ("total_tokens", ctypes.c_int64), ("alpha", ctypes.c_float),
                 ("ln_eps", ctypes.c_float), ("rel_bias_len", ctypes.c_int32),
                 ("time_bias_len", ctypes.c_int32), ("time_bucket_div", ctypes.c_double),
-                ("dtype", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+                ("dtype", ctypes.c_int32), ("flags", ctypes.c_int32)]
+
+# mask variants (Params.flags)
+FLAG_CTX_SEES_HISTORY, FLAG_REL_ABS = 0x1, 0x2
 
 
 _lib = None
@@ -112,14 +115,15 @@ def dtype_code(t: torch.Tensor) -> int:
 
 
 def make_params(q, v, seq_offsets, *, alpha, max_seqlen, max_attn_len=0, rel_bias=None,
-                time_bias=None, time_bucket_div=0.301, ln_eps=1e-5) -> Params:
+                time_bias=None, time_bucket_div=0.301, ln_eps=1e-5, mask_flags=0) -> Params:
     T, H, dqk = q.shape
     return Params(batch=seq_offsets.numel() - 1, num_heads=H, d_qk=dqk, d_v=v.shape[2],
                   max_seqlen=int(max_seqlen), max_attn_len=int(max_attn_len), total_tokens=T,
                   alpha=float(alpha), ln_eps=float(ln_eps),
                   rel_bias_len=0 if rel_bias is None else rel_bias.numel(),
                   time_bias_len=0 if time_bias is None else time_bias.numel(),
-                  time_bucket_div=float(time_bucket_div), dtype=dtype_code(q), reserved=0)
+                  time_bucket_div=float(time_bucket_div), dtype=dtype_code(q),
+                  flags=int(mask_flags))
 
 
 def fwd_workspace_size(params: Params) -> int:
@@ -145,12 +149,12 @@ class Saved:
 
 def fwd(q, k, v, u, seq_offsets, num_contextuals=None, num_targets=None, timestamps=None,
         rel_bias=None, time_bias=None, *, alpha, max_seqlen, max_attn_len=0,
-        time_bucket_div=0.301, ln_eps=1e-5, training=False, out=None, workspace=None,
-        saved: Optional[Saved] = None, stream=None):
+        time_bucket_div=0.301, ln_eps=1e-5, mask_flags=0, training=False, out=None,
+        workspace=None, saved: Optional[Saved] = None, stream=None):
     """out [T, H*d_v] (and Saved(y, mean, rstd) when training)."""
     p = make_params(q, v, seq_offsets, alpha=alpha, max_seqlen=max_seqlen,
                     max_attn_len=max_attn_len, rel_bias=rel_bias, time_bias=time_bias,
-                    time_bucket_div=time_bucket_div, ln_eps=ln_eps)
+                    time_bucket_div=time_bucket_div, ln_eps=ln_eps, mask_flags=mask_flags)
     T, H, dv = v.shape
     dev = q.device
     if out is None:
@@ -174,11 +178,12 @@ def fwd(q, k, v, u, seq_offsets, num_contextuals=None, num_targets=None, timesta
 
 def bwd(dout, q, k, v, u, seq_offsets, num_contextuals=None, num_targets=None, timestamps=None,
         rel_bias=None, time_bias=None, *, saved: Saved, alpha, max_seqlen, max_attn_len=0,
-        time_bucket_div=0.301, ln_eps=1e-5, grads=None, workspace=None, stream=None):
+        time_bucket_div=0.301, ln_eps=1e-5, mask_flags=0, grads=None, workspace=None,
+        stream=None):
     """(dq, dk, dv, du, d_rel_bias or None, d_time_bias or None)."""
     p = make_params(q, v, seq_offsets, alpha=alpha, max_seqlen=max_seqlen,
                     max_attn_len=max_attn_len, rel_bias=rel_bias, time_bias=time_bias,
-                    time_bucket_div=time_bucket_div, ln_eps=ln_eps)
+                    time_bucket_div=time_bucket_div, ln_eps=ln_eps, mask_flags=mask_flags)
     dev = q.device
     if grads is None:
         grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v),
@@ -286,7 +291,8 @@ def batch_to_device(b, device="cuda"):
 
 def batch_kwargs(b):
     return dict(alpha=b.alpha, max_seqlen=b.max_seqlen, max_attn_len=b.max_attn_len,
-                time_bucket_div=b.time_bucket_div, ln_eps=b.ln_eps)
+                time_bucket_div=b.time_bucket_div, ln_eps=b.ln_eps,
+                mask_flags=int(getattr(b, "mask_flags", 0)))
 
 
 def run_fwd(b, dev_tensors=None, training=False, **kw):

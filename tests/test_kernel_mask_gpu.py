@@ -30,7 +30,7 @@ def _params(lengths, W):
     return ops.Params(batch=len(lengths), num_heads=1, d_qk=64, d_v=64, max_seqlen=max(lengths),
                       max_attn_len=W, total_tokens=int(sum(lengths)), alpha=1.0, ln_eps=1e-5,
                       rel_bias_len=0, time_bias_len=0, time_bucket_div=0.301,
-                      dtype=ops.HSTU_BF16, reserved=0)
+                      dtype=ops.HSTU_BF16, flags=0)
 
 
 def _device_batch(seqs):

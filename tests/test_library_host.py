@@ -43,7 +43,7 @@ def test_status_strings_and_version():
 def _params(**kw):
     base = dict(batch=2, num_heads=2, d_qk=32, d_v=32, max_seqlen=16, max_attn_len=0,
                 total_tokens=20, alpha=0.5, ln_eps=1e-5, rel_bias_len=17, time_bias_len=128,
-                time_bucket_div=0.301, dtype=ops.HSTU_BF16, reserved=0)
+                time_bucket_div=0.301, dtype=ops.HSTU_BF16, flags=0)
     base.update(kw)
     return ops.Params(**base)
 
@@ -54,7 +54,7 @@ def test_workspace_size_and_validation():
     assert n >= 256 + 20 * 64 * 4
     assert ops.bwd_workspace_size(p) >= 256 + 20 * 64 * 4 + 20 * 64 * 4
     for bad in [dict(num_heads=0), dict(d_qk=0), dict(d_v=300), dict(max_seqlen=0),
-                dict(time_bias_len=-1), dict(dtype=7), dict(reserved=1),
+                dict(time_bias_len=-1), dict(dtype=7), dict(flags=4),
                 dict(time_bucket_div=0.0), dict(batch=-1)]:
         with pytest.raises(ops.HstuError) as e:
             ops.fwd_workspace_size(_params(**bad))

@@ -153,7 +153,7 @@ def test_debug_mask_bit_exact(W):
     p = ops.Params(batch=len(lengths), num_heads=1, d_qk=16, d_v=16, max_seqlen=max(lengths),
                    max_attn_len=W, total_tokens=int(offs[-1]), alpha=1.0, ln_eps=1e-5,
                    rel_bias_len=0, time_bias_len=0, time_bucket_div=0.301, dtype=ops.HSTU_BF16,
-                   reserved=0)
+                   flags=0)
     for s, L in enumerate(lengths):
         got = ops.debug_mask(p, d_offs, d_ctx, d_tgt, s, L).numpy()
         ref, _ = oracle.mask(L, int(ctx[s]), int(tgt[s]), W)
@@ -515,3 +515,57 @@ def test_a_wait_that_runs_out_is_reported_and_the_context_stays_usable():
     finally:
         ops.set_wait_test(0, stall=False)
     _fwd_bwd_check(b, "after the stall test")
+
+
+# ------------------------------------------------------------------ mask variants
+#
+# Contextual rows that see the whole history (flag 1) and the rel index |p(i) - p(j)| (flag 2),
+# through both tensor-core kernels and the CUDA-core path: values against the oracle, and
+# the tensor-core kernels' masked-pair structure bit for bit.
+
+VARIANT_CASES = [
+    # name, lengths, H, dqk, dv, dtype, ctx, tgt, W, R, NB
+    ("bf16-family", [5, 200, 77, 260, 129], 2, 128, 128, "bf16", [1, 4, 0, 8, 3],
+     [2, 20, 5, 0, 64], 0, 261, 128),
+    ("bf16-window", [700, 130, 2, 256], 2, 64, 64, "bf16", [8, 40, 1, 130], [32, 0, 1, 60], 100,
+     101, 128),
+    ("bf16-all-targets", [64, 150], 2, 64, 64, "bf16", [0, 3], [64, 100], 0, 10, 128),
+    ("f32-family", [5, 200, 77], 2, 32, 48, "f32", [1, 4, 3], [2, 20, 5], 9, 40, 64),
+]
+
+
+@pytest.mark.parametrize("flags", [1, 2, 3])
+@pytest.mark.parametrize("case", VARIANT_CASES, ids=[c[0] for c in VARIANT_CASES])
+def test_mask_variants_fwd_bwd_parity(case, flags):
+    name, lengths, H, dqk, dv, dtype, ctx, tgt, W, R, NB = case
+    b = synth.make_batch(np.random.default_rng(90 + flags), lengths, H, dqk, dv, dtype,
+                         contextuals=ctx, targets=tgt, max_attn_len=W, rel_bias_len=R,
+                         time_bias_len=NB, with_dout=True, mask_flags=flags)
+    _fwd_bwd_check(b, "%s flags=%d" % (name, flags))
+
+
+@pytest.mark.parametrize("flags", [1, 3])
+def test_mask_variants_kernel_mask_bit_exact(flags):
+    seqs = [(1, 1, 0), (33, 5, 3), (129, 40, 32), (300, 130, 60), (257, 129, 127), (70, 0, 70)]
+    lengths = [q[0] for q in seqs]
+    offs = np.zeros(len(seqs) + 1, np.int64)
+    offs[1:] = np.cumsum(lengths)
+    d_offs = torch.from_numpy(offs).cuda()
+    d_ctx = torch.tensor([q[1] for q in seqs], dtype=torch.int32, device="cuda")
+    d_tgt = torch.tensor([q[2] for q in seqs], dtype=torch.int32, device="cuda")
+    for W in (0, 33):
+        p = ops.Params(batch=len(seqs), num_heads=1, d_qk=64, d_v=64, max_seqlen=max(lengths),
+                       max_attn_len=W, total_tokens=int(offs[-1]), alpha=1.0, ln_eps=1e-5,
+                       rel_bias_len=0, time_bias_len=0, time_bucket_div=0.301,
+                       dtype=ops.HSTU_BF16, flags=flags)
+        for s, (L, c, t) in enumerate(seqs):
+            pad = (L + 127) // 128 * 128
+            ref = oracle.mask_rows(L, c, t, W, 0, pad, pad, flags).astype(bool)
+            for kernel in ("fwd", "bwd"):
+                got = ops.debug_kernel_mask(p, d_offs, d_ctx, d_tgt, s, kernel, 0, pad,
+                                            pad).numpy()
+                assert np.array_equal(got[:L, :L], ref[:L, :L]), (kernel, L, c, t, W, flags)
+                if kernel == "fwd":
+                    assert not got[:L, L:].any()
+                else:
+                    assert not got[L:, :L].any()
