@@ -493,3 +493,66 @@ def test_mask_variants_backward_finite_differences(flags):
                          rel_bias_len=12, time_bias_len=32, mask_flags=flags)
     dout = np.random.default_rng(80 + flags).standard_normal(b.u.shape)
     _fd_check(b, dout, samples=8)
+
+
+# ---------------------------------------------------------------- jagged operations
+
+def _read_sl_golden(path):
+    g = {}
+    for ln in open(path):
+        ln = ln.split("#")[0].strip()
+        if ln:
+            k, *v = ln.split()
+            g[k] = v
+    return g
+
+
+def test_stochastic_length_hand_example(golden_dir):
+    from oracle import jagged
+    g = _read_sl_golden(f"{golden_dir}/stochastic_length_example.txt")
+    lengths = [int(x) for x in g["lengths"]]
+    offs = np.concatenate([[0], np.cumsum(lengths)])
+    rows, new = jagged.stochastic_length(offs, [int(x) for x in g["contextuals"]],
+                                         [int(x) for x in g["targets"]],
+                                         [float(x) for x in g["keys"]], int(g["budget"][0]))
+    assert rows.tolist() == [int(x) for x in g["rows"]]
+    assert new.tolist() == [int(x) for x in g["offsets"]]
+
+
+def test_stochastic_length_invariants():
+    """Kept counts, order, what is always kept, and that the kept history keys are the
+    smallest ones; a budget at least the history keeps everything."""
+    from oracle import jagged
+    rng = np.random.default_rng(5)
+    L = rng.integers(0, 60, size=40)
+    c = np.minimum(rng.integers(0, 4, size=40), L)
+    t = np.minimum(rng.integers(0, 6, size=40), L - c)
+    offs = np.concatenate([[0], np.cumsum(L)])
+    keys = rng.integers(0, 8, size=int(offs[-1])) / 8.0          # many ties
+    for budget in (0, 5, 17, 1000):
+        rows, new = jagged.stochastic_length(offs, c, t, keys, budget)
+        for b in range(40):
+            a, e = offs[b], offs[b + 1]
+            E = e - t[b]
+            mine = rows[new[b]:new[b + 1]] - a
+            assert np.all(np.diff(mine) > 0)                        # original order
+            h = E - a - c[b]
+            assert len(mine) == c[b] + t[b] + min(h, budget)
+            assert set(range(c[b])) <= set(mine) and set(range(E - a, e - a)) <= set(mine)
+            kept = [j for j in mine if c[b] <= j < E - a]
+            dropped = [j for j in range(c[b], E - a) if j not in set(mine)]
+            if kept and dropped:   # every kept (key, pos) precedes every dropped one
+                assert max((keys[a + j], j) for j in kept) < min((keys[a + j], j) for j in dropped)
+        if budget == 1000:
+            assert rows.tolist() == list(range(int(offs[-1])))
+
+
+def test_jagged_concat_and_gather_examples():
+    from oracle import jagged
+    a = np.arange(6).reshape(3, 2); oa = np.array([0, 1, 1, 3])
+    b = 10 + np.arange(8).reshape(4, 2); ob = np.array([0, 2, 3, 4])
+    v, o = jagged.jagged_concat([(a, oa), (b, ob)])
+    assert o.tolist() == [0, 3, 4, 7]
+    assert v[:, 0].tolist() == [0, 10, 12, 14, 2, 4, 16]
+    g = jagged.gather_rows(b, [3, 0, 0])
+    assert g[:, 0].tolist() == [16, 10, 10]
