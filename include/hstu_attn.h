@@ -92,6 +92,12 @@ typedef enum { HSTU_F32 = 0, HSTU_BF16 = 1 } hstu_dtype_t;
 /* Mask variants (params->flags). */
 #define HSTU_FLAG_CTX_SEES_HISTORY 0x1   /* contextual rows attend to every non-candidate key */
 #define HSTU_FLAG_REL_ABS          0x2   /* rel index min(|p(i) - p(j)|, R - 1) */
+/* Forward (inference) only: compute the query tiles that hold candidate rows (rows >= E) and
+ * skip the others, whose rows of out are then unspecified.  With target-group masking a
+ * candidate's output depends only on the history and itself, so candidates can be scored in
+ * micro-batches appended to a cached history ("Scaling HSTU: ragged execution, candidate
+ * amortization and content features", "Many candidates make reuse valuable": M-FALCON). */
+#define HSTU_FLAG_CANDIDATES_ONLY  0x4
 
 /* Bits of the device status word. */
 #define HSTU_DEV_BAD_OFFSETS   0x1   /* seq_offsets not non-decreasing / not ending at T */
@@ -247,6 +253,47 @@ hstu_status_t hstu_attn_set_stage_events(int32_t stage, void *start_event, void 
  * Process-wide and not thread-safe: for tests only.
  */
 hstu_status_t hstu_attn_set_wait_test(int64_t limit_cycles, int32_t stall);
+
+/*
+ * Stochastic Length ("Scaling HSTU: ragged execution, candidate amortization and content
+ * features", "Variable length is a central systems issue": it samples sequence lengths in
+ * training).  Reading (the page gives no formula): sequence b keeps its contextual prefix
+ * (num_contextuals[b] tokens) and candidates (the last num_targets[b]), and of its h history
+ * tokens the min(h, budget) whose keys are smallest, the earlier position first on equal
+ * keys, all in their original order.  keys [total_tokens] fp32 (device, no NaN) are the
+ * caller's random numbers, one per token (history tokens' keys are read).  Writes
+ * out_offsets [batch + 1] (device, int64; the new jagged offsets) and out_rows (device,
+ * int64, room for total_tokens): the kept rows as indices into the input rows, sequence by
+ * sequence; hstu_gather_rows then gathers any per-token tensor.  A sequence with invalid
+ * offsets or counts keeps nothing and sets a HSTU_DEV_* bit in *status (device int32,
+ * NULL = not reported).  Enqueued on `stream`; allocates nothing.
+ */
+hstu_status_t hstu_stochastic_length(const int64_t *seq_offsets, const int32_t *num_contextuals,
+                                     const int32_t *num_targets, int32_t batch,
+                                     int64_t total_tokens, const float *keys, int32_t budget,
+                                     int64_t *out_rows, int64_t *out_offsets, int32_t *status,
+                                     void *stream);
+
+/*
+ * dst row r = src row rows[r] for r < min(*n_rows, max_rows); rows of row_bytes bytes.  rows
+ * and n_rows (a count, e.g. the last entry of jagged offsets) are device memory, read on the
+ * device; max_rows bounds the work from the host.  Indices must lie inside src.
+ */
+hstu_status_t hstu_gather_rows(const void *src, int64_t row_bytes, const int64_t *rows,
+                               const int64_t *n_rows, int64_t max_rows, void *dst, void *stream);
+
+/*
+ * Jagged concatenation ("HSTU-MUSA: HSTU for Moore Threads (MUSA)", "Project Structure":
+ * jagged tensor concatenation): n_parts (1..16) jagged tensors of the same row width
+ * row_bytes, part q given by values[q] and offsets[q] ([batch + 1], device), become one whose
+ * sequence b holds the rows of part 0's sequence b, then part 1's, ...  values and offsets
+ * are host arrays of device pointers; out_offsets [batch + 1] (device) receives the sums of
+ * the parts' offsets, out_values room for all rows.  E.g. contextual, history and candidate
+ * tokens into one sequence per user.
+ */
+hstu_status_t hstu_jagged_concat(int32_t n_parts, const void *const *values,
+                                 const int64_t *const *offsets, int32_t batch, int64_t row_bytes,
+                                 void *out_values, int64_t *out_offsets, void *stream);
 
 /* Static description of a status code. */
 const char *hstu_status_string(hstu_status_t status);

@@ -5,4 +5,4 @@ include/hstu_attn.h).  `ops` is its thin Python binding; `synth` draws seeded in
 `accounting` counts valid pairs, FLOPs and bytes.  Nothing here computes the method on
 the CPU: without the built library (or without a GPU) the binding raises.
 """
-__all__ = ["ops", "synth", "accounting"]
+__all__ = ["ops", "synth", "accounting", "shard", "mfalcon"]

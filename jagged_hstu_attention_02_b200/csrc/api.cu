@@ -65,7 +65,8 @@ const ThrEntry &thresholds(double div, int nb)
 hstu_status_t validate(const hstu_attn_params_t *p)
 {
     if (!p) return HSTU_ERR_INVALID_ARGUMENT;
-    if (p->flags & ~(HSTU_FLAG_CTX_SEES_HISTORY | HSTU_FLAG_REL_ABS)) return HSTU_ERR_INVALID_ARGUMENT;
+    if (p->flags & ~(HSTU_FLAG_CTX_SEES_HISTORY | HSTU_FLAG_REL_ABS | HSTU_FLAG_CANDIDATES_ONLY))
+        return HSTU_ERR_INVALID_ARGUMENT;
     if (p->batch < 0 || p->num_heads < 1 || p->total_tokens < 0) return HSTU_ERR_INVALID_ARGUMENT;
     if (p->max_seqlen < 1) return HSTU_ERR_INVALID_ARGUMENT;
     if (p->d_qk < 1 || p->d_v < 1 || p->d_qk > 256 || p->d_v > 256)
@@ -253,6 +254,7 @@ hstu_status_t hstu_attn_fwd(const hstu_attn_params_t *p, const void *q, const vo
     const bool train = saved_y != nullptr;
     if (train != (saved_mean != nullptr) || train != (saved_rstd != nullptr))
         return HSTU_ERR_INVALID_ARGUMENT;
+    if (train && (p->flags & HSTU_FLAG_CANDIDATES_ONLY)) return HSTU_ERR_UNSUPPORTED;
     if (!workspace || !seq_offsets) return HSTU_ERR_INVALID_ARGUMENT;
     if (p->total_tokens > 0 && (!q || !k || !v || !u || !out)) return HSTU_ERR_INVALID_ARGUMENT;
     if (p->rel_bias_len > 0 && !rel_bias) return HSTU_ERR_INVALID_ARGUMENT;
@@ -303,6 +305,7 @@ hstu_status_t hstu_attn_bwd(const hstu_attn_params_t *p, const void *dout, const
 {
     hstu_status_t st = validate(p);
     if (st != HSTU_OK) return st;
+    if (p->flags & HSTU_FLAG_CANDIDATES_ONLY) return HSTU_ERR_UNSUPPORTED;   // forward only
     if (!workspace || !seq_offsets) return HSTU_ERR_INVALID_ARGUMENT;
     if (p->total_tokens > 0 &&
         (!dout || !q || !k || !v || !u || !saved_y || !saved_mean || !saved_rstd || !dq || !dk ||
@@ -419,6 +422,53 @@ hstu_status_t hstu_attn_debug_kernel_mask(const hstu_attn_params_t *p,
                                   nullptr, nullptr);
     HSTU_CUDA_TRY(launch_debug_kernel_mask(d, seq, kernel, row_begin, row_count, key_count, bits,
                                            reinterpret_cast<cudaStream_t>(stream)));
+    return HSTU_OK;
+}
+
+hstu_status_t hstu_stochastic_length(const int64_t *seq_offsets, const int32_t *num_contextuals,
+                                     const int32_t *num_targets, int32_t batch,
+                                     int64_t total_tokens, const float *keys, int32_t budget,
+                                     int64_t *out_rows, int64_t *out_offsets, int32_t *status,
+                                     void *stream)
+{
+    if (batch < 0 || batch > 65535 || total_tokens < 0 || budget < 0 || !seq_offsets ||
+        !out_offsets || (total_tokens > 0 && (!keys || !out_rows)))
+        return HSTU_ERR_INVALID_ARGUMENT;
+    DevParams d;
+    std::memset(&d, 0, sizeof(d));
+    d.B = batch;
+    d.T = total_tokens;
+    d.N = INT32_MAX;          // no length limit here
+    d.offsets = seq_offsets;
+    d.ctx = num_contextuals;
+    d.tgt = num_targets;
+    d.status = status;
+    HSTU_CUDA_TRY(launch_stochastic_length(d, keys, budget, out_rows, out_offsets,
+                                           reinterpret_cast<cudaStream_t>(stream)));
+    return HSTU_OK;
+}
+
+hstu_status_t hstu_gather_rows(const void *src, int64_t row_bytes, const int64_t *rows,
+                               const int64_t *n_rows, int64_t max_rows, void *dst, void *stream)
+{
+    if (row_bytes <= 0 || max_rows < 0 || !n_rows || (max_rows > 0 && (!src || !rows || !dst)))
+        return HSTU_ERR_INVALID_ARGUMENT;
+    HSTU_CUDA_TRY(launch_gather_rows(src, row_bytes, rows, n_rows, max_rows, dst,
+                                     reinterpret_cast<cudaStream_t>(stream)));
+    return HSTU_OK;
+}
+
+hstu_status_t hstu_jagged_concat(int32_t n_parts, const void *const *values,
+                                 const int64_t *const *offsets, int32_t batch, int64_t row_bytes,
+                                 void *out_values, int64_t *out_offsets, void *stream)
+{
+    if (n_parts < 1 || n_parts > kMaxConcatParts || batch < 0 || row_bytes <= 0 || !values ||
+        !offsets || !out_values || !out_offsets)
+        return HSTU_ERR_INVALID_ARGUMENT;
+    for (int q = 0; q < n_parts; ++q)
+        if (!values[q] || !offsets[q]) return HSTU_ERR_INVALID_ARGUMENT;
+    HSTU_CUDA_TRY(launch_jagged_concat(n_parts, values, offsets, batch, row_bytes, out_values,
+                                       out_offsets, reinterpret_cast<cudaStream_t>(stream)));
     return HSTU_OK;
 }
 

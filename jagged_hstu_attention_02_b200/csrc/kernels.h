@@ -114,6 +114,17 @@ bool encode_tmap_bf16(CUtensorMap *m, const void *base, int d, int H, int64_t T)
 
 cudaError_t launch_debug_mask(const DevParams &p, int seq, int seq_len, uint32_t *bits,
                               cudaStream_t st);
+
+// Jagged operations (jagged.cu).  p carries B, T, offsets, counts and the status word.
+constexpr int kMaxConcatParts = 16;
+cudaError_t launch_stochastic_length(const DevParams &p, const float *keys, int budget,
+                                     int64_t *out_rows, int64_t *out_offsets, cudaStream_t st);
+cudaError_t launch_gather_rows(const void *src, int64_t row_bytes, const int64_t *rows,
+                               const int64_t *n_rows, int64_t max_rows, void *dst,
+                               cudaStream_t st);
+cudaError_t launch_jagged_concat(int n_parts, const void *const *values,
+                                 const int64_t *const *offsets, int B, int64_t row_bytes,
+                                 void *out, int64_t *out_offsets, cudaStream_t st);
 // Mask of rows [row0, row0 + nrows) x keys [0, nkeys) (nkeys a multiple of 32) of sequence
 // seq as the tensor-core forward (kernel 0) or backward (kernel 1) decides it.
 cudaError_t launch_debug_kernel_mask(const DevParams &p, int seq, int kernel, int row0,

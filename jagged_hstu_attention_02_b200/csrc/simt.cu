@@ -101,6 +101,7 @@ __global__ void __launch_bounds__(kThreads)
     }
     const int i0 = qt * kFwdBM;
     if (i0 >= s.L) return;
+    if ((p.flags & HSTU_FLAG_CANDIDATES_ONLY) && i0 + kFwdBM <= s.E) return;   // no candidate row
     const int tid = threadIdx.x, ty = tid / 16, tx = tid % 16;
 
     load_header(p, hd);

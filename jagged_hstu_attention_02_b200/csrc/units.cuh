@@ -85,6 +85,9 @@ struct UnitFeed {
         decode(x);
         if (!seq_may_have_tile(p, b, tile)) return false;
         s = load_seq(p, b, false);
+        // the forward in candidates-only mode skips query tiles without a candidate row
+        if (!ASCENDING && (p.flags & HSTU_FLAG_CANDIDATES_ONLY) && (tile + 1) * TILE <= s.E)
+            return false;
         return tile * TILE < s.L;
     }
 

@@ -11,6 +11,7 @@ import os
 from dataclasses import dataclass
 from typing import Optional
 
+import numpy as np
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -24,6 +25,7 @@ DEV_BAD_OFFSETS, DEV_BAD_COUNTS, DEV_SEQ_TOO_LONG, DEV_WAIT_TIMEOUT = 0x1, 0x2, 
 EXPORTED = ["hstu_attn_fwd_workspace_size", "hstu_attn_fwd", "hstu_attn_bwd_workspace_size",
             "hstu_attn_bwd", "hstu_attn_read_device_status", "hstu_attn_debug_mask",
             "hstu_attn_debug_kernel_mask", "hstu_attn_set_wait_test",
+            "hstu_stochastic_length", "hstu_gather_rows", "hstu_jagged_concat",
             "hstu_attn_time_thresholds", "hstu_attn_set_stage_events", "hstu_status_string",
             "hstu_attn_version"]
 STAGES = {"fwd_attn": 0, "fwd_norm": 1, "bwd_norm": 2, "bwd_attn": 3}
@@ -45,7 +47,7 @@ class Params(ctypes.Structure):
                 ("dtype", ctypes.c_int32), ("flags", ctypes.c_int32)]
 
 # mask variants (Params.flags)
-FLAG_CTX_SEES_HISTORY, FLAG_REL_ABS = 0x1, 0x2
+FLAG_CTX_SEES_HISTORY, FLAG_REL_ABS, FLAG_CANDIDATES_ONLY = 0x1, 0x2, 0x4
 
 
 _lib = None
@@ -75,6 +77,12 @@ def lib():
                                                 ctypes.POINTER(ctypes.c_uint64)]
         L.hstu_attn_set_stage_events.argtypes = [ctypes.c_int32, _VP, _VP]
         L.hstu_attn_set_wait_test.argtypes = [ctypes.c_int64, ctypes.c_int32]
+        L.hstu_stochastic_length.argtypes = [_VP, _VP, _VP, ctypes.c_int32, ctypes.c_int64, _VP,
+                                             ctypes.c_int32, _VP, _VP, _VP, _VP]
+        L.hstu_gather_rows.argtypes = [_VP, ctypes.c_int64, _VP, _VP, ctypes.c_int64, _VP, _VP]
+        L.hstu_jagged_concat.argtypes = [ctypes.c_int32, ctypes.POINTER(_VP),
+                                         ctypes.POINTER(_VP), ctypes.c_int32, ctypes.c_int64,
+                                         _VP, _VP, _VP]
         L.hstu_status_string.restype = ctypes.c_char_p
         L.hstu_status_string.argtypes = [ctypes.c_int]
         L.hstu_attn_version.restype = ctypes.c_int32
@@ -264,6 +272,54 @@ def set_wait_test(limit_cycles: int = 0, stall: bool = False):
            "hstu_attn_set_wait_test")
 
 
+# ------------------------------------------------------------------ jagged operations
+
+MAX_CONCAT_PARTS = 16
+
+def stochastic_length(seq_offsets, num_contextuals, num_targets, keys, budget: int,
+                      status=None, stream=None):
+    """(kept rows [T] int64 (first new_offsets[-1] valid), new offsets [B+1] int64)."""
+    T = int(keys.numel())
+    B = seq_offsets.numel() - 1
+    rows = torch.empty(max(T, 1), dtype=torch.int64, device=seq_offsets.device)
+    offs = torch.empty(B + 1, dtype=torch.int64, device=seq_offsets.device)
+    _check(lib().hstu_stochastic_length(_ptr(seq_offsets), _ptr(num_contextuals),
+                                        _ptr(num_targets), B, T, _ptr(keys), int(budget),
+                                        _ptr(rows), _ptr(offs), _ptr(status), _stream(stream)),
+           "hstu_stochastic_length")
+    return rows, offs
+
+
+def gather_rows(src, rows, n_rows, max_rows: int, out=None, stream=None):
+    """out[r] = src[rows[r]] for r < n_rows (a device scalar tensor), up to max_rows rows."""
+    if out is None:
+        out = torch.empty((max_rows,) + tuple(src.shape[1:]), dtype=src.dtype, device=src.device)
+    row_bytes = src[0].numel() * src.element_size() if src.numel() else 1
+    _check(lib().hstu_gather_rows(_ptr(src), row_bytes, _ptr(rows), _ptr(n_rows), int(max_rows),
+                                  _ptr(out), _stream(stream)), "hstu_gather_rows")
+    return out
+
+
+def jagged_concat(parts, out=None, stream=None):
+    """parts: list of (values [T_q, ...], offsets [B+1]); (values, offsets) of the per-sequence
+    concatenation."""
+    vals0, offs0 = parts[0]
+    B = offs0.numel() - 1
+    total = sum(int(v.shape[0]) for v, _ in parts)
+    if out is None:
+        out = torch.empty((total,) + tuple(vals0.shape[1:]), dtype=vals0.dtype,
+                          device=vals0.device)
+    out_offs = torch.empty(B + 1, dtype=torch.int64, device=offs0.device)
+    n = len(parts)
+    V = (_VP * n)(*[_ptr(v) for v, _ in parts])
+    O = (_VP * n)(*[_ptr(o) for _, o in parts])
+    row_bytes = vals0[0].numel() * vals0.element_size() if vals0.numel() else \
+        int(np.prod(vals0.shape[1:])) * vals0.element_size()
+    _check(lib().hstu_jagged_concat(n, V, O, B, row_bytes, _ptr(out), _ptr(out_offs),
+                                    _stream(stream)), "hstu_jagged_concat")
+    return out, out_offs
+
+
 def version() -> int:
     return int(lib().hstu_attn_version())
 
@@ -297,15 +353,19 @@ def batch_kwargs(b):
 
 def run_fwd(b, dev_tensors=None, training=False, **kw):
     t = batch_to_device(b) if dev_tensors is None else dev_tensors
+    args = batch_kwargs(b)
+    args.update(kw)
     return fwd(t["q"], t["k"], t["v"], t["u"], t["seq_offsets"], t["num_contextuals"],
                t["num_targets"], t["timestamps"], t["rel_bias"], t["time_bias"],
-               training=training, **batch_kwargs(b), **kw)
+               training=training, **args)
 
 
 def run_bwd(b, saved, dout=None, dev_tensors=None, **kw):
     t = batch_to_device(b) if dev_tensors is None else dev_tensors
     if dout is None:
         dout = t["dout"]
+    args = batch_kwargs(b)
+    args.update(kw)
     return bwd(dout, t["q"], t["k"], t["v"], t["u"], t["seq_offsets"], t["num_contextuals"],
                t["num_targets"], t["timestamps"], t["rel_bias"], t["time_bias"], saved=saved,
-               **batch_kwargs(b), **kw)
+               **args)

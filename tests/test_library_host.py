@@ -54,7 +54,7 @@ def test_workspace_size_and_validation():
     assert n >= 256 + 20 * 64 * 4
     assert ops.bwd_workspace_size(p) >= 256 + 20 * 64 * 4 + 20 * 64 * 4
     for bad in [dict(num_heads=0), dict(d_qk=0), dict(d_v=300), dict(max_seqlen=0),
-                dict(time_bias_len=-1), dict(dtype=7), dict(flags=4),
+                dict(time_bias_len=-1), dict(dtype=7), dict(flags=8),
                 dict(time_bucket_div=0.0), dict(batch=-1)]:
         with pytest.raises(ops.HstuError) as e:
             ops.fwd_workspace_size(_params(**bad))

@@ -556,3 +556,42 @@ def test_jagged_concat_and_gather_examples():
     assert v[:, 0].tolist() == [0, 10, 12, 14, 2, 4, 16]
     g = jagged.gather_rows(b, [3, 0, 0])
     assert g[:, 0].tolist() == [16, 10, 10]
+
+
+def test_candidate_outputs_do_not_depend_on_the_other_candidates():
+    """The property M-FALCON rests on ("Scaling HSTU", "Many candidates make reuse valuable"):
+    under target-group masking a candidate's output, computed with the history plus only
+    some of the candidates (same N), equals its output in the full batch, and the history
+    rows equal those of the history alone.  Exact in fp64: the same terms in the same order."""
+    import dataclasses
+    rng = np.random.default_rng(31)
+    H, d = 2, 8
+    hist_len = [12, 30, 5]
+    ncand = [7, 3, 4]
+    full = synth.make_batch(rng, [h + c for h, c in zip(hist_len, ncand)], H, d, d, "f32",
+                            contextuals=[2, 3, 1], targets=ncand, max_attn_len=6,
+                            rel_bias_len=40, time_bias_len=32)
+    ref = oracle.fwd(full)
+    N = full.max_seqlen
+    offs = full.seq_offsets
+
+    def sub(keep_cands):
+        rows, lens, tg = [], [], []
+        for s in range(3):
+            a = offs[s]
+            rows += list(range(a, a + hist_len[s]))
+            sel = [a + hist_len[s] + j for j in keep_cands[s]]
+            rows += sel
+            lens.append(hist_len[s] + len(sel))
+            tg.append(len(sel))
+        rows = np.array(rows)
+        o = np.concatenate([[0], np.cumsum(lens)])
+        return rows, dataclasses.replace(
+            full, seq_offsets=o, num_targets=np.array(tg, np.int32), q=full.q[rows],
+            k=full.k[rows], v=full.v[rows], u=full.u[rows], timestamps=full.timestamps[rows],
+            max_seqlen=N)
+
+    for keep in ([[], [], []], [[0, 2], [1], [3]], [[6], [0, 1, 2], []]):
+        rows, b = sub(keep)
+        got = oracle.fwd(b)["out"]
+        assert np.array_equal(got, ref["out"][rows])
