@@ -595,3 +595,47 @@ def test_candidate_outputs_do_not_depend_on_the_other_candidates():
         rows, b = sub(keep)
         got = oracle.fwd(b)["out"]
         assert np.array_equal(got, ref["out"][rows])
+
+
+# ---------------------------------------------------------------- the layer around the path
+
+def test_fused_projection_splits_into_four_projections():
+    """One projection with columns U | V | Q | K (head-major) equals four separate
+    projections, with d_qk != d_v; the SiLU variant applies to every branch."""
+    from oracle import layer
+    rng = np.random.default_rng(7)
+    T, dm, H, dqk, dv = 9, 16, 3, 4, 6
+    x = rng.standard_normal((T, dm))
+    Wu, Wv = rng.standard_normal((dm, H * dv)), rng.standard_normal((dm, H * dv))
+    Wq, Wk = rng.standard_normal((dm, H * dqk)), rng.standard_normal((dm, H * dqk))
+    bu, bv, bq, bk = (rng.standard_normal(w.shape[1]) for w in (Wu, Wv, Wq, Wk))
+    W = np.concatenate([Wu, Wv, Wq, Wk], axis=1)
+    bias = np.concatenate([bu, bv, bq, bk])
+    silu = lambda a: a / (1 + np.exp(-a))
+    for act, f in ((False, lambda a: a), (True, silu)):
+        u, v, q, k = layer.uvqk(x, W, bias, H, dqk, dv, silu=act)
+        assert np.allclose(u, f(x @ Wu + bu))
+        assert np.allclose(v[:, 2, :], f(x @ Wv + bv)[:, 2 * dv:3 * dv])
+        assert np.allclose(q[:, 1, :], f(x @ Wq + bq)[:, dqk:2 * dqk])
+        assert np.allclose(k.reshape(T, -1), f(x @ Wk + bk))
+
+
+def test_layer_output_projection_and_residual():
+    """W_o = 0 and no bias: the layer returns its input (the residual).  W_o the identity
+    (d_model = H * d_v), no residual: it returns the attention output."""
+    from oracle import layer
+    b = synth.make_batch(np.random.default_rng(8), [7, 12], 2, 4, 4, "f32", contextuals=1,
+                         targets=[2, 3], rel_bias_len=13, time_bias_len=16)
+    dm = 8
+    rng = np.random.default_rng(9)
+    x = rng.standard_normal((b.total_tokens, dm))
+    W = rng.standard_normal((dm, 2 * 2 * 4 + 2 * 2 * 4)) * 0.3
+    r0 = layer.layer_fwd(b, x, W, None, np.zeros((dm, dm)), None)
+    assert np.array_equal(r0["o"], x)
+    r1 = layer.out_proj(r0["attn"], np.eye(dm), None, None)
+    assert np.allclose(r1, r0["attn"])
+    # the input normalisation: mean 0 and variance var/(var + eps) per token
+    xn = layer.layer_norm(x, 1e-5)
+    assert np.allclose(xn.mean(1), 0, atol=1e-12)
+    v = x.var(1)
+    assert np.allclose(xn.var(1), v / (v + 1e-5))
