@@ -255,6 +255,35 @@ hstu_status_t hstu_attn_set_stage_events(int32_t stage, void *start_event, void 
 hstu_status_t hstu_attn_set_wait_test(int64_t limit_cycles, int32_t stall);
 
 /*
+ * The layer around the attention ("HSTU tensor by tensor: SiLU aggregation, temporal bias and
+ * gating": "Similar shape, different aggregation", o_i = W_o[U_i (.) Norm(sum_j A_ij V_j)] + x_i;
+ * "Trace four projections": normalised inputs produce U/V/Q/K through one larger projection
+ * split to match the weight layout).  bf16 tensors, fp32 biases, row-major, 16-byte aligned
+ * device pointers; each call enqueues kernels on `stream` and allocates nothing.  status
+ * (device int32, may be NULL) receives HSTU_DEV_WAIT_TIMEOUT if a bounded wait gave up.
+ *
+ * hstu_layer_norm_rows: y = LayerNorm(x) per row of `width` (multiple of 32, <= 1024) values,
+ * no affine (biased variance, eps inside the square root): the input normalisation.
+ *
+ * hstu_uvqk_proj: [T, N] = x [T, d_model] w [d_model, N] (+ bias [N]) (SiLU of every value when
+ * silu = 1), N = 2 H (d_v + d_qk), columns ordered U | V | Q | K, each head-major; written as
+ * u [T, H*d_v], v [T, H, d_v], q [T, H, d_qk], k [T, H, d_qk] -- the layouts hstu_attn_fwd
+ * takes.  d_model, H*d_v and H*d_qk must be multiples of 64.
+ *
+ * hstu_out_proj: out [T, d_model] = z [T, d_in] w_o [d_in, d_model] (+ bias [d_model]) (+ x
+ * [T, d_model], the residual; NULL for none).  d_in and d_model multiples of 64.
+ */
+hstu_status_t hstu_layer_norm_rows(const void *x, void *y, int64_t rows, int32_t width,
+                                   float eps, void *stream);
+hstu_status_t hstu_uvqk_proj(const void *x, const void *w, const float *bias, int64_t tokens,
+                             int32_t d_model, int32_t num_heads, int32_t d_qk, int32_t d_v,
+                             int32_t silu, void *u, void *v, void *q, void *k, int32_t *status,
+                             void *stream);
+hstu_status_t hstu_out_proj(const void *z, const void *w_o, const float *bias, const void *x,
+                            int64_t tokens, int32_t d_in, int32_t d_model, void *out,
+                            int32_t *status, void *stream);
+
+/*
  * Stochastic Length ("Scaling HSTU: ragged execution, candidate amortization and content
  * features", "Variable length is a central systems issue": it samples sequence lengths in
  * training).  Reading (the page gives no formula): sequence b keeps its contextual prefix

@@ -425,6 +425,58 @@ hstu_status_t hstu_attn_debug_kernel_mask(const hstu_attn_params_t *p,
     return HSTU_OK;
 }
 
+hstu_status_t hstu_layer_norm_rows(const void *x, void *y, int64_t rows, int32_t width,
+                                   float eps, void *stream)
+{
+    if (rows < 0 || width < 32 || width > 1024 || width % 32 != 0 || !(eps >= 0.f) ||
+        (rows > 0 && (!x || !y)))
+        return HSTU_ERR_INVALID_ARGUMENT;
+    HSTU_CUDA_TRY(launch_ln_rows(x, y, rows, width, eps, reinterpret_cast<cudaStream_t>(stream)));
+    return HSTU_OK;
+}
+
+hstu_status_t hstu_uvqk_proj(const void *x, const void *w, const float *bias, int64_t tokens,
+                             int32_t d_model, int32_t num_heads, int32_t d_qk, int32_t d_v,
+                             int32_t silu, void *u, void *v, void *q, void *k, int32_t *status,
+                             void *stream)
+{
+    if (tokens < 0 || tokens > INT32_MAX || d_model < 64 || d_model % 64 != 0 || num_heads < 1 ||
+        d_qk < 1 || d_v < 1 || ((int64_t)num_heads * d_qk) % 64 != 0 ||
+        ((int64_t)num_heads * d_v) % 64 != 0 || (silu != 0 && silu != 1))
+        return HSTU_ERR_INVALID_ARGUMENT;
+    const int64_t N = 2 * (int64_t)num_heads * (d_v + d_qk);
+    if (N > 65536) return HSTU_ERR_UNSUPPORTED;
+    if (tokens == 0) return HSTU_OK;
+    const void *ptrs[] = {x, w, bias, u, v, q, k};
+    for (int x_ = 0; x_ < 7; ++x_)
+        if ((x_ != 2 && !ptrs[x_]) || !aligned16(ptrs[x_])) return HSTU_ERR_INVALID_ARGUMENT;
+    const int hv = num_heads * d_v, hq = num_heads * d_qk;
+    const int lo[5] = {0, hv, 2 * hv, 2 * hv + hq, 2 * hv + 2 * hq};
+    void *outs[4] = {u, v, q, k};
+    HSTU_CUDA_TRY(launch_gemm(x, w, (int)tokens, (int)N, d_model, bias, silu != 0, nullptr, 4, lo,
+                              outs, status, g_wait_limit, reinterpret_cast<cudaStream_t>(stream)));
+    return HSTU_OK;
+}
+
+hstu_status_t hstu_out_proj(const void *z, const void *w_o, const float *bias, const void *x,
+                            int64_t tokens, int32_t d_in, int32_t d_model, void *out,
+                            int32_t *status, void *stream)
+{
+    if (tokens < 0 || tokens > INT32_MAX || d_in < 64 || d_in % 64 != 0 || d_model < 64 ||
+        d_model % 64 != 0 || d_model > 65536)
+        return HSTU_ERR_INVALID_ARGUMENT;
+    if (tokens == 0) return HSTU_OK;
+    const void *ptrs[] = {z, w_o, bias, x, out};
+    for (int x_ = 0; x_ < 5; ++x_)
+        if (((x_ == 0 || x_ == 1 || x_ == 4) && !ptrs[x_]) || !aligned16(ptrs[x_]))
+            return HSTU_ERR_INVALID_ARGUMENT;
+    const int lo[2] = {0, d_model};
+    void *outs[1] = {out};
+    HSTU_CUDA_TRY(launch_gemm(z, w_o, (int)tokens, d_model, d_in, bias, false, x, 1, lo, outs,
+                              status, g_wait_limit, reinterpret_cast<cudaStream_t>(stream)));
+    return HSTU_OK;
+}
+
 hstu_status_t hstu_stochastic_length(const int64_t *seq_offsets, const int32_t *num_contextuals,
                                      const int32_t *num_targets, int32_t batch,
                                      int64_t total_tokens, const float *keys, int32_t budget,

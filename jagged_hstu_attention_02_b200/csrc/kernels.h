@@ -115,6 +115,15 @@ bool encode_tmap_bf16(CUtensorMap *m, const void *base, int d, int H, int64_t T)
 cudaError_t launch_debug_mask(const DevParams &p, int seq, int seq_len, uint32_t *bits,
                               cudaStream_t st);
 
+// The layer around the attention (gemm.cu): C = A B (+ bias, SiLU, residual), bf16, with the
+// columns [seg_lo[s], seg_lo[s+1]) of C written to outs[s]; and the input LayerNorm.
+cudaError_t launch_gemm(const void *A, const void *B, int M, int N, int K, const float *bias,
+                        bool silu, const void *resid, int nseg, const int *seg_lo,
+                        void *const *outs, int32_t *status, long long wait_limit,
+                        cudaStream_t st);
+cudaError_t launch_ln_rows(const void *x, void *y, int64_t rows, int width, float eps,
+                           cudaStream_t st);
+
 // Jagged operations (jagged.cu).  p carries B, T, offsets, counts and the status word.
 constexpr int kMaxConcatParts = 16;
 cudaError_t launch_stochastic_length(const DevParams &p, const float *keys, int budget,

@@ -26,6 +26,7 @@ EXPORTED = ["hstu_attn_fwd_workspace_size", "hstu_attn_fwd", "hstu_attn_bwd_work
             "hstu_attn_bwd", "hstu_attn_read_device_status", "hstu_attn_debug_mask",
             "hstu_attn_debug_kernel_mask", "hstu_attn_set_wait_test",
             "hstu_stochastic_length", "hstu_gather_rows", "hstu_jagged_concat",
+            "hstu_layer_norm_rows", "hstu_uvqk_proj", "hstu_out_proj",
             "hstu_attn_time_thresholds", "hstu_attn_set_stage_events", "hstu_status_string",
             "hstu_attn_version"]
 STAGES = {"fwd_attn": 0, "fwd_norm": 1, "bwd_norm": 2, "bwd_attn": 3}
@@ -79,6 +80,12 @@ def lib():
         L.hstu_attn_set_wait_test.argtypes = [ctypes.c_int64, ctypes.c_int32]
         L.hstu_stochastic_length.argtypes = [_VP, _VP, _VP, ctypes.c_int32, ctypes.c_int64, _VP,
                                              ctypes.c_int32, _VP, _VP, _VP, _VP]
+        L.hstu_layer_norm_rows.argtypes = [_VP, _VP, ctypes.c_int64, ctypes.c_int32,
+                                           ctypes.c_float, _VP]
+        L.hstu_uvqk_proj.argtypes = [_VP, _VP, _VP, ctypes.c_int64] + [ctypes.c_int32] * 5 + \
+            [_VP] * 6
+        L.hstu_out_proj.argtypes = [_VP, _VP, _VP, _VP, ctypes.c_int64, ctypes.c_int32,
+                                    ctypes.c_int32, _VP, _VP, _VP]
         L.hstu_gather_rows.argtypes = [_VP, ctypes.c_int64, _VP, _VP, ctypes.c_int64, _VP, _VP]
         L.hstu_jagged_concat.argtypes = [ctypes.c_int32, ctypes.POINTER(_VP),
                                          ctypes.POINTER(_VP), ctypes.c_int32, ctypes.c_int64,
@@ -318,6 +325,58 @@ def jagged_concat(parts, out=None, stream=None):
     _check(lib().hstu_jagged_concat(n, V, O, B, row_bytes, _ptr(out), _ptr(out_offs),
                                     _stream(stream)), "hstu_jagged_concat")
     return out, out_offs
+
+
+# ------------------------------------------------------------------ the layer around the path
+
+def layer_norm_rows(x, eps=1e-5, out=None, stream=None):
+    """LayerNorm (no affine) of every row of the bf16 matrix x."""
+    if out is None:
+        out = torch.empty_like(x)
+    _check(lib().hstu_layer_norm_rows(_ptr(x), _ptr(out), x.shape[0], x.shape[1], float(eps),
+                                      _stream(stream)), "hstu_layer_norm_rows")
+    return out
+
+
+def uvqk_proj(x, w, bias, num_heads, d_qk, d_v, silu=False, status=None, stream=None):
+    """(u [T, H*d_v], v [T,H,d_v], q [T,H,d_qk], k [T,H,d_qk]) of the fused projection."""
+    T = x.shape[0]
+    dev, dt = x.device, x.dtype
+    u = torch.empty((T, num_heads * d_v), dtype=dt, device=dev)
+    v = torch.empty((T, num_heads, d_v), dtype=dt, device=dev)
+    q = torch.empty((T, num_heads, d_qk), dtype=dt, device=dev)
+    k = torch.empty((T, num_heads, d_qk), dtype=dt, device=dev)
+    _check(lib().hstu_uvqk_proj(_ptr(x), _ptr(w), _ptr(bias), T, x.shape[1], num_heads, d_qk,
+                                d_v, 1 if silu else 0, _ptr(u), _ptr(v), _ptr(q), _ptr(k),
+                                _ptr(status), _stream(stream)), "hstu_uvqk_proj")
+    return u, v, q, k
+
+
+def out_proj(z, w_o, bias=None, x=None, status=None, stream=None):
+    """z [T, d_in] w_o [d_in, d_model] (+ bias) (+ x): the output projection and residual."""
+    T, d_model = z.shape[0], w_o.shape[1]
+    out = torch.empty((T, d_model), dtype=z.dtype, device=z.device)
+    _check(lib().hstu_out_proj(_ptr(z), _ptr(w_o), _ptr(bias), _ptr(x), T, z.shape[1], d_model,
+                               _ptr(out), _ptr(status), _stream(stream)), "hstu_out_proj")
+    return out
+
+
+def layer_fwd(x, seq_offsets, num_contextuals, num_targets, timestamps, rel_bias, time_bias,
+              w_uvqk, b_uvqk, w_o, b_o, *, num_heads, d_qk, d_v, alpha, max_seqlen,
+              max_attn_len=0, time_bucket_div=0.301, ln_eps=1e-5, mask_flags=0,
+              uvqk_silu=False, stream=None):
+    """One HSTU layer on jagged tokens x [T, d_model] (bf16): input LayerNorm, fused U/V/Q/K
+    projection, attention with LayerNorm and U gating, output projection with bias and the
+    residual.  Returns dict(xn, u, v, q, k, attn, o)."""
+    xn = layer_norm_rows(x, ln_eps, stream=stream)
+    u, v, q, k = uvqk_proj(xn, w_uvqk, b_uvqk, num_heads, d_qk, d_v, silu=uvqk_silu,
+                           stream=stream)
+    attn = fwd(q, k, v, u, seq_offsets, num_contextuals, num_targets, timestamps, rel_bias,
+               time_bias, alpha=alpha, max_seqlen=max_seqlen, max_attn_len=max_attn_len,
+               time_bucket_div=time_bucket_div, ln_eps=ln_eps, mask_flags=mask_flags,
+               stream=stream)
+    o = out_proj(attn, w_o, b_o, x, stream=stream)
+    return dict(xn=xn, u=u, v=v, q=q, k=k, attn=attn, o=o)
 
 
 def version() -> int:
