@@ -328,6 +328,7 @@ def run_ours(args, world, rank, local):
         for cfg in FWD_BLOCKS:
             blocks[FWD_BLOCKS[cfg][0]] = measure_fwd_block(ops, torch, peaks, peak_kind, cfg,
                                                            args, with_cpu=not args.no_cpu)
+        blocks["layer_projections"] = measure_layer_block(ops, torch, peaks, peak_kind, args)
     cpu = cpu_baseline_train(b) if (rank == 0 and world == 1 and not args.no_cpu) else None
     if world > 1:
         torch.distributed.barrier()
@@ -553,6 +554,56 @@ def measure_fwd_block(ops, torch, peaks, peak_kind, cfg, args, with_cpu=True):
     return blk
 
 
+def measure_layer_block(ops, torch, peaks, peak_kind, args, d_model=128):
+    """The dense steps of the layer around the attention on the MovieLens-shaped tokens
+    (d_model 128, 4 heads of 128): the fused U/V/Q/K projection and the output projection
+    with residual, each timed alone (>= 50 L2-flushed calls, median) against HBM (their
+    arithmetic intensity is below the ridge point)."""
+    b = synth.make_config(1)
+    T, H, d = b.total_tokens, b.num_heads, b.d_qk
+    N = 4 * H * d
+    g = torch.Generator(device="cuda").manual_seed(7)
+    x = torch.randn((T, d_model), device="cuda", generator=g).to(torch.bfloat16)
+    w = (torch.randn((d_model, N), device="cuda", generator=g) / d_model ** 0.5).to(torch.bfloat16)
+    bw = torch.randn(N, device="cuda", generator=g) * 0.1
+    z = torch.randn((T, H * d), device="cuda", generator=g).to(torch.bfloat16)
+    wo = (torch.randn((H * d, d_model), device="cuda", generator=g) / (H * d) ** 0.5).to(torch.bfloat16)
+    bo = torch.randn(d_model, device="cuda", generator=g) * 0.1
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    iters = max(50, args.steps)
+    res = {}
+    cases = {
+        "uvqk_proj": (lambda: ops.uvqk_proj(x, w, bw, H, d, d),
+                      2 * T * d_model + 2 * d_model * N + 4 * N + 2 * T * N, 2 * T * d_model * N),
+        "out_proj": (lambda: ops.out_proj(z, wo, bo, x),
+                     2 * T * H * d + 2 * H * d * d_model + 4 * d_model + 4 * T * d_model,
+                     2 * T * H * d * d_model),
+    }
+    for name, (fn, byts, fl) in cases.items():
+        for _ in range(max(args.warmup, 3)):
+            fn()
+        times = []
+        for _ in range(iters):
+            flush.fill_(1.0)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            e1.synchronize()
+            times.append(e0.elapsed_time(e1))
+        ms = statistics.median(times)
+        gbs = byts / (ms * 1e-3) / 1e9
+        res[name] = {"ms": round(ms, 4), "tflops": round(fl / (ms * 1e-3) / 1e12, 2),
+                     "roofline": {"bound": "hbm", "achieved": round(gbs, 1),
+                                  "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                  "frac": round(gbs / peaks["hbm_gbs"], 4),
+                                  "algorithmic_bytes": byts, "peak_source": peak_kind}}
+    return {"workload": "layer around the attention on the MovieLens-shaped tokens "
+                        "(T=%d, d_model=%d, H=%d, d=%d), bf16" % (T, d_model, H, d),
+            "iters": iters, "timing": "median of CUDA-event times, L2 flushed before each call",
+            "gpu_launches": 2 * iters, **res}
+
+
 def _timed_sample(b, run, target_s):
     """Times `run` (the oracle, parallel over sequences) on a sample of b's first sequences:
     one sequence first; if that is quick, as many sequences as the oracle has threads, then
@@ -657,7 +708,15 @@ def main():
     ap.add_argument("--fwd-only", type=int, default=None, metavar="WORKLOAD",
                     help="only the inference-forward block of this workload (1, 2 or 3), "
                          "without CPU baseline (for profiling its kernel)")
+    ap.add_argument("--layer-only", action="store_true",
+                    help="only the layer-projection block (for profiling its GEMMs)")
     args = ap.parse_args()
+    if args.layer_only:
+        import torch
+        from jagged_hstu_attention_02_b200 import ops
+        peaks, kind = load_peaks()
+        print(json.dumps(measure_layer_block(ops, torch, peaks, kind, args)), flush=True)
+        return
     if args.fwd_only is not None:
         import torch
         from jagged_hstu_attention_02_b200 import ops

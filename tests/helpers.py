@@ -1,4 +1,6 @@
 """Shared test helpers: tolerances and row selection (data handling only)."""
+import os
+
 import numpy as np
 
 from jagged_hstu_attention_02_b200.synth import sub_batch  # noqa: F401
@@ -19,6 +21,10 @@ def assert_close(got, ref, dtype, what=""):
     err, scale = max_err(got, ref)
     rel, ab = TOL[dtype]
     tol = rel * scale + ab
+    log = os.environ.get("HSTU_PARITY_LOG")
+    if log:   # margin record: what, max|err|, tolerance, their ratio
+        with open(log, "a") as f:
+            f.write("%s\t%.4e\t%.4e\t%.4f\n" % (what, err, tol, err / tol if tol else 0.0))
     assert np.all(np.isfinite(np.asarray(got, dtype=np.float64))), what + ": non-finite values"
     assert err <= tol, "%s: max|err| %.3e > tol %.3e (max|ref| %.3e)" % (what, err, tol, scale)
     return err, scale
