@@ -224,6 +224,15 @@ __device__ __forceinline__ void fwd_quarter(const FwdEpi &e, const HalfTime &ht,
     }
 }
 
+// Byte permute of x with sign replication: selector nibble 8 + k gives byte k's top bit
+// repeated over a byte (0x9988: bytes 0 and 1 to halves 0 and 1; 0xBBAA: bytes 2 and 3).
+__device__ __forceinline__ uint32_t sign_bytes(uint32_t x, uint32_t sel)
+{
+    uint32_t d;
+    asm("prmt.b32 %0, %1, 0, %2;" : "=r"(d) : "r"(x), "r"(sel));
+    return d;
+}
+
 __device__ __forceinline__ uint32_t add_bf16x2(uint32_t a, uint32_t b)
 {
     uint32_t d;
@@ -241,6 +250,23 @@ __device__ __forceinline__ void inf_chunk(const FwdEpi &e, const HalfTime &ht, u
                                           uint32_t tlo2, uint32_t thi2, uint32_t a1,
                                           uint32_t span, uint32_t (&a)[4])
 {
+    // the 8 keys' stamps (relative to the quarter's minimum) in two 16-byte loads
+    int32_t tk[8];
+    if (TM == 1 || TM == 2) {
+        const int4 x0 = *reinterpret_cast<const int4 *>(e.tk32 + cb);
+        const int4 x1 = *reinterpret_cast<const int4 *>(e.tk32 + cb + 4);
+        tk[0] = x0.x; tk[1] = x0.y; tk[2] = x0.z; tk[3] = x0.w;
+        tk[4] = x1.x; tk[5] = x1.y; tk[6] = x1.z; tk[7] = x1.w;
+    }
+    // the keys' valid bits moved to the sign bits of bytes: key 4h + b -> bit 7 of byte b of
+    // z[h] (a multiply by 2^7 + 2^14 + 2^21 + 2^28 places non-overlapping copies of the 4
+    // bits), so that one byte permute with sign replication gives a pair's half masks
+    uint32_t z[2] = {0u, 0u};
+    if (!FULL) {
+        const uint32_t v8 = vmask >> cb;
+        z[0] = (v8 & 0xFu) * 0x10204080u;
+        z[1] = ((v8 >> 4) & 0xFu) * 0x10204080u;
+    }
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
         const int c = cb + 2 * q;
@@ -257,14 +283,14 @@ __device__ __forceinline__ void inf_chunk(const FwdEpi &e, const HalfTime &ht, u
         if (TM == 0) {
             t2 = tlo2;
         } else if (TM == 1) {
-            const bool h0 = (uint32_t)e.tk32[c] - a1 >= span;
-            const bool h1 = (uint32_t)e.tk32[c + 1] - a1 >= span;
+            const bool h0 = (uint32_t)tk[2 * q] - a1 >= span;
+            const bool h1 = (uint32_t)tk[2 * q + 1] - a1 >= span;
             t2 = ((h0 ? thi2 : tlo2) & 0x0000FFFFu) | ((h1 ? thi2 : tlo2) & 0xFFFF0000u);
         } else if (TM == 2) {
             float v[2];
 #pragma unroll
             for (int k = 0; k < 2; ++k) {
-                const int32_t d = ht.t_rel - e.tk32[c + k];
+                const int32_t d = ht.t_rel - tk[2 * q + k];
                 uint32_t dt = (uint32_t)(d < 0 ? -d : d);
                 dt = min(dt, (uint32_t)INT32_MAX - 1u);
                 const float tv = e.tbh[lut_bucket(e.lut, dt)];
@@ -279,9 +305,7 @@ __device__ __forceinline__ void inf_chunk(const FwdEpi &e, const HalfTime &ht, u
         const uint32_t s2 = pack_bf16x2(__uint_as_float(s[2 * q]), __uint_as_float(s[2 * q + 1]));
         const uint32_t h2 = add_bf16x2(fma_bf16x2(ha2, s2, r2), t2);
         uint32_t a2 = fma_bf16x2(h2, tanh_bf16x2(h2), h2);
-        if (!FULL)
-            a2 &= (((vmask >> c) & 1u) ? 0x0000FFFFu : 0u) |
-                  (((vmask >> (c + 1)) & 1u) ? 0xFFFF0000u : 0u);
+        if (!FULL) a2 &= sign_bytes(z[q >> 1], (q & 1) ? 0xBBAAu : 0x9988u);
         a[q] = a2;
     }
 }
