@@ -172,8 +172,9 @@ hstu_status_t hstu_attn_debug_mask(const hstu_attn_params_t *params, const int64
                                    int32_t seq, int32_t seq_len, uint32_t *bits, void *stream);
 
 /*
- * Test hook: the mask of sequence `seq` as the tensor-core kernels decide it (bf16 inputs,
- * d_qk and d_v in {64, 128}): a pair is valid when the kernel visits its 128 x 128 tile and
+ * Test hook: the mask of sequence `seq` as the tensor-core kernels decide it (bf16 inputs;
+ * the forward for any admitted head dims, the backward for d_qk and d_v in {64, 128}): a
+ * pair is valid when the kernel visits its 128 x 128 tile and
  * the 32-wide block the pair lies in marks it.  kernel = 0 selects the forward's decisions
  * (per query row and 32-key block), kernel = 1 the backward's (per key and 32-query block).
  * Writes rows [row_begin, row_begin + row_count) x keys [0, key_count) of the mask, row-major,

@@ -891,7 +891,10 @@ cudaError_t launch_bwd(const BwdTcArgs &a, cudaStream_t st)
 
 }  // namespace
 
-bool tc_bwd_supported(int dqk, int dv, int64_t T) { return tc_fwd_supported(dqk, dv, T); }
+bool tc_bwd_supported(int dqk, int dv, int64_t T)
+{
+    return (dqk == 64 || dqk == 128) && (dv == 64 || dv == 128) && T < ((int64_t)1 << 31);
+}
 
 cudaError_t launch_tc_bwd(const DevParams &p, const void *q, const void *k, const void *v,
                           const void *dy_bf16, float *dq_acc, void *dk, void *dv, float *d_rel,

@@ -783,10 +783,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                                         __uint_as_float(ro[4 * x + 3]) * p.inv_N);
                 transpose_chunks<NCH>(yc);
                 const int j = lane % NCH, r0 = i - j;         // rows r0 .. r0 + NCH - 1
-                float *yb = args.y + (s.start + r0) * (int64_t)p.D + un.h * DV + wq * OC + 4 * j;
+                // (head dims below DV run padded: only the first p.dv columns are real)
+                const int col = wq * OC + 4 * j;
+                float *yb = args.y + (s.start + r0) * (int64_t)p.D + un.h * p.dv + col;
 #pragma unroll
                 for (int c = 0; c < NCH; ++c)
-                    if (r0 + c < s.L)
+                    if (r0 + c < s.L && col < p.dv)
                         *reinterpret_cast<float4 *>(yb + (int64_t)c * p.D) = yc[c];
             }
             ++n;
@@ -873,9 +875,13 @@ bool encode_tmap_bf16(CUtensorMap *m, const void *base, int d, int H, int64_t T)
     return r == CUDA_SUCCESS;
 }
 
+// Head dims: multiples of 16 up to 128.  Below 64 (or between 64 and 128) the kernel for 64
+// (128) runs on zero-padded tiles: the TMA boxes past d read zeros, which add nothing to
+// Q K^T, and the output columns past d_v are not stored.
 bool tc_fwd_supported(int dqk, int dv, int64_t T)
 {
-    return (dqk == 64 || dqk == 128) && (dv == 64 || dv == 128) && T < ((int64_t)1 << 31);
+    return dqk >= 16 && dqk <= 128 && dqk % 16 == 0 && dv >= 16 && dv <= 128 && dv % 16 == 0 &&
+           T < ((int64_t)1 << 31);
 }
 
 cudaError_t launch_tc_fwd(const DevParams &p, const void *q, const void *k, const void *v,
@@ -891,11 +897,11 @@ cudaError_t launch_tc_fwd(const DevParams &p, const void *q, const void *k, cons
     if (!encode_tmap_bf16(&a.tq, q, p.dqk, p.H, p.T) || !encode_tmap_bf16(&a.tk, k, p.dqk, p.H, p.T) ||
         !encode_tmap_bf16(&a.tv, v, p.dv, p.H, p.T))
         return cudaErrorInvalidValue;
-    if (p.dqk == 128 && p.dv == 128) return launch_tc<128, 128>(a, training, st);
-    if (p.dqk == 128 && p.dv == 64) return launch_tc<128, 64>(a, training, st);
-    if (p.dqk == 64 && p.dv == 128) return launch_tc<64, 128>(a, training, st);
-    if (p.dqk == 64 && p.dv == 64) return launch_tc<64, 64>(a, training, st);
-    return cudaErrorInvalidValue;
+    const int dq = p.dqk <= 64 ? 64 : 128, dvp = p.dv <= 64 ? 64 : 128;   // padded dims
+    if (dq == 128 && dvp == 128) return launch_tc<128, 128>(a, training, st);
+    if (dq == 128 && dvp == 64) return launch_tc<128, 64>(a, training, st);
+    if (dq == 64 && dvp == 128) return launch_tc<64, 128>(a, training, st);
+    return launch_tc<64, 64>(a, training, st);
 }
 
 }  // namespace hstu

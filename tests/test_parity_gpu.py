@@ -51,6 +51,9 @@ SMALL_CASES = [
     ("bf16-all-targets", [64, 150], 2, 64, 64, "bf16", 0, [64, 150], 0, 10, 128),
     ("bf16-all-context", [64, 150], 2, 64, 64, "bf16", [64, 150], 0, 0, 151, 128),
     ("bf16-dqk-ne-dv", [90, 300], 2, 128, 64, "bf16", 1, 3, 0, 301, 128),
+    # head dims the tensor-core forward runs zero-padded to 64 / 128
+    ("bf16-d96-d48", [33, 260, 129], 2, 96, 48, "bf16", [1, 4, 0], [2, 9, 1], 0, 261, 128),
+    ("bf16-d16-d112", [150, 7, 300], 3, 16, 112, "bf16", 2, [3, 0, 30], 60, 61, 128),
 ]
 
 
@@ -61,6 +64,19 @@ def test_fwd_parity_small(case):
                          contextuals=ctx, targets=tgt, max_attn_len=W, rel_bias_len=R,
                          time_bias_len=NB)
     _fwd_check(b, what=name)
+
+
+BF16_CASES = [c for c in SMALL_CASES if c[5] == "bf16"]
+
+
+@pytest.mark.parametrize("case", BF16_CASES, ids=[c[0] for c in BF16_CASES])
+def test_fwd_parity_small_inference(case):
+    """The inference forward (bf16 pair arithmetic in the epilogue) on the small shapes."""
+    name, lengths, H, dqk, dv, dtype, ctx, tgt, W, R, NB = case
+    b = synth.make_batch(np.random.default_rng(102), lengths, H, dqk, dv, dtype,
+                         contextuals=ctx, targets=tgt, max_attn_len=W, rel_bias_len=R,
+                         time_bias_len=NB)
+    _fwd_check(b, training=False, what=name + " inference")
 
 
 @pytest.mark.parametrize("case", SMALL_CASES, ids=[c[0] for c in SMALL_CASES])
