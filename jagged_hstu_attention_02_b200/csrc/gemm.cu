@@ -11,8 +11,9 @@
 // fp32 accumulation in TMEM.  Persistent CTAs take 128 x BN output tiles in a static order;
 // warp 0 lane 0 streams 64-wide K slices of A and B through a four-stage ring with TMA
 // (128-byte swizzle), warp 1 lane 0 issues tcgen05.mma into one of two TMEM accumulators,
-// warps 2-5 read the other accumulator back (thread = row = TMEM lane) and write bf16
-// outputs, so a tile's epilogue overlaps the next tile's MMAs.  Every wait is bounded.
+// warps 2-9 read the other accumulator back (two warps per TMEM lane quarter, each half of
+// the columns; thread = row = TMEM lane) and write bf16 outputs, so a tile's epilogue
+// overlaps the next tile's MMAs.  Every wait is bounded.
 #include <cudaTypedefs.h>
 
 #include <cstring>
@@ -30,7 +31,9 @@ namespace {
 constexpr int GBM = 128;          // rows (tokens) per tile
 constexpr int GBK = 64;           // K per stage: one 128-byte swizzle atom of bf16
 constexpr int kGStages = 4;
-constexpr int kGThreads = 192;    // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue (warp 2: TMEM)
+constexpr int kGEpiWarps = 8;
+constexpr int kGThreads = 32 * (2 + kGEpiWarps);   // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue
+                                                   // (warp 2 also owns TMEM)
 constexpr int kMaxSegs = 4;
 
 struct GemmArgs {
@@ -85,8 +88,8 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_tc_kernel(const __grid_cons
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     if (threadIdx.x == 0) {
         for (int x = 0; x < G_NBARS; ++x) mbar_init(&bars[x], 1);
-        mbar_init(&bars[ACC_EMPTY], 4);
-        mbar_init(&bars[ACC_EMPTY + 1], 4);
+        mbar_init(&bars[ACC_EMPTY], kGEpiWarps);
+        mbar_init(&bars[ACC_EMPTY + 1], kGEpiWarps);
         fence_mbar_init();
     }
     if (warp == 2) tmem_alloc(slot, 2 * BN);
@@ -171,8 +174,14 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_tc_kernel(const __grid_cons
         }
     } else {
         // -------------------------------------------------------------------- epilogue
-        const int r = (warp & 3) * 32 + lane;          // row of the tile == TMEM lane
-        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        // 64 columns per step: a lane converts its row's 64 values into 8 chunks of 8 bf16,
+        // then a transpose over groups of 8 lanes lets 8 lanes store one row's 128 bytes
+        // side by side (segment boundaries and N are multiples of 64)
+        const int q = warp & 3;                          // TMEM lane quarter: rows 32q ..
+        const int half = (warp - 2) >> 2;                // columns [half BN/2, (half+1) BN/2)
+        const int r = q * 32 + lane;                     // row of the tile == TMEM lane
+        const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+        const int j = lane & 7;                          // chunk this lane stores
         int t = 0;
         bool ok = true;
         for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++t) {
@@ -185,53 +194,66 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_tc_kernel(const __grid_cons
             tc_fence_after();
             const int m = m0 + r;
 #pragma unroll 1
-            for (int c0 = 0; c0 < BN; c0 += 32) {
-                __syncwarp();                             // the warp-wide TMEM load below
-                uint32_t v[32];
+            for (int c0 = half * (BN / 2); c0 < (half + 1) * (BN / 2); c0 += 64) {
+                __syncwarp();                             // the warp-wide TMEM loads below
+                uint32_t v[32], w[32];
                 tmem_ld32(tmem + lane_base + acc * BN + c0, v);
+                tmem_ld32(tmem + lane_base + acc * BN + c0 + 32, w);
                 tmem_wait_ld();
                 reg_fence(v);
+                reg_fence(w);
                 const int nb = n0 + c0;
-                if (nb < a.N && m < a.M) {
+                if (nb >= a.N) continue;                  // (warp-uniform)
                 int sg = 0;
                 while (sg + 1 < a.nseg && nb >= a.lo[sg + 1]) ++sg;
-                float f[32];
+                float4 o[8];                              // 8 chunks of 8 bf16 (as 16 bytes)
 #pragma unroll
-                for (int x = 0; x < 32; ++x) f[x] = __uint_as_float(v[x]);
-                if (a.bias) {
-                    const float4 *bp = reinterpret_cast<const float4 *>(a.bias + nb);
+                for (int hh = 0; hh < 2; ++hh) {
+                    float f[32];
 #pragma unroll
-                    for (int x = 0; x < 8; ++x) {
-                        const float4 bv = __ldg(bp + x);
-                        f[4 * x] += bv.x; f[4 * x + 1] += bv.y; f[4 * x + 2] += bv.z; f[4 * x + 3] += bv.w;
-                    }
-                }
-                if (a.silu) {
+                    for (int x = 0; x < 32; ++x) f[x] = __uint_as_float(hh ? w[x] : v[x]);
+                    const int nc = nb + 32 * hh;
+                    if (a.bias) {
+                        const float4 *bp = reinterpret_cast<const float4 *>(a.bias + nc);
 #pragma unroll
-                    for (int x = 0; x < 32; ++x) f[x] = f[x] * __fdividef(1.0f, 1.0f + __expf(-f[x]));
-                }
-                if (a.resid) {
-                    const uint4 *rp = reinterpret_cast<const uint4 *>(a.resid + (int64_t)m * a.N + nb);
-#pragma unroll
-                    for (int x = 0; x < 4; ++x) {
-                        const uint4 rv = rp[x];
-                        const uint32_t w[4] = {rv.x, rv.y, rv.z, rv.w};
-#pragma unroll
-                        for (int y = 0; y < 4; ++y) {
-                            f[8 * x + 2 * y] += __uint_as_float(w[y] << 16);
-                            f[8 * x + 2 * y + 1] += __uint_as_float(w[y] & 0xFFFF0000u);
+                        for (int x = 0; x < 8; ++x) {
+                            const float4 bv = __ldg(bp + x);
+                            f[4 * x] += bv.x; f[4 * x + 1] += bv.y; f[4 * x + 2] += bv.z; f[4 * x + 3] += bv.w;
                         }
                     }
-                }
-                const int width = a.lo[sg + 1] - a.lo[sg];
-                uint4 *op = reinterpret_cast<uint4 *>(a.out[sg] + (int64_t)m * width + (nb - a.lo[sg]));
+                    if (a.silu) {
 #pragma unroll
-                for (int x = 0; x < 4; ++x)
-                    op[x] = make_uint4(pack_bf16x2(f[8 * x], f[8 * x + 1]),
-                                       pack_bf16x2(f[8 * x + 2], f[8 * x + 3]),
-                                       pack_bf16x2(f[8 * x + 4], f[8 * x + 5]),
-                                       pack_bf16x2(f[8 * x + 6], f[8 * x + 7]));
+                        for (int x = 0; x < 32; ++x) f[x] = f[x] * __fdividef(1.0f, 1.0f + __expf(-f[x]));
+                    }
+                    if (a.resid && m < a.M) {
+                        const uint4 *rp = reinterpret_cast<const uint4 *>(a.resid + (int64_t)m * a.N + nc);
+#pragma unroll
+                        for (int x = 0; x < 4; ++x) {
+                            const uint4 rv = rp[x];
+                            const uint32_t u4[4] = {rv.x, rv.y, rv.z, rv.w};
+#pragma unroll
+                            for (int y = 0; y < 4; ++y) {
+                                f[8 * x + 2 * y] += __uint_as_float(u4[y] << 16);
+                                f[8 * x + 2 * y + 1] += __uint_as_float(u4[y] & 0xFFFF0000u);
+                            }
+                        }
+                    }
+#pragma unroll
+                    for (int x = 0; x < 4; ++x)
+                        o[4 * hh + x] = make_float4(__uint_as_float(pack_bf16x2(f[8 * x], f[8 * x + 1])),
+                                                    __uint_as_float(pack_bf16x2(f[8 * x + 2], f[8 * x + 3])),
+                                                    __uint_as_float(pack_bf16x2(f[8 * x + 4], f[8 * x + 5])),
+                                                    __uint_as_float(pack_bf16x2(f[8 * x + 6], f[8 * x + 7])));
                 }
+                // lane l now stores chunk j = l % 8 of rows l - j .. l - j + 7 of this warp
+                transpose_chunks<8>(o);
+                const int width = a.lo[sg + 1] - a.lo[sg];
+                const int mr = m0 + q * 32 + (lane - j);
+                __nv_bfloat16 *ob = a.out[sg] + (int64_t)mr * width + (nb - a.lo[sg]) + 8 * j;
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    if (mr + c < a.M)
+                        *reinterpret_cast<float4 *>(ob + (int64_t)c * width) = o[c];
             }
             __syncwarp();
             tc_fence_before();
