@@ -36,6 +36,7 @@ from jagged_hstu_attention_02_b200 import accounting, synth  # noqa: E402
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 << 20
 WORKLOAD_CFG = 4          # MovieLens-shaped inputs + upstream gradient
+METRIC = "jagged HSTU attn fwd+bwd TFLOP/s (valid pairs) on 1 B200"
 # inference-forward blocks: workload -> (block name, roofline that bounds its attention kernel)
 FWD_BLOCKS = {2: ("long_history_fwd", "tensor"), 3: ("windowed_fwd", "tensor"),
               1: ("movielens_fwd", "hbm")}
@@ -336,7 +337,7 @@ def run_ours(args, world, rank, local):
     if rank != 0:
         return
     line = {
-        "metric": "jagged HSTU attn fwd+bwd TFLOP/s (valid pairs) on 1 B200",
+        "metric": METRIC,
         "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
@@ -684,7 +685,7 @@ def run_reference(args, world, rank):
               ("all" if k == 1 else "every %d-th sequence:" % k, b.batch, full.batch,
                b.total_tokens))
     line = {"impl": "reference",
-            "metric": "jagged HSTU attn fwd+bwd TFLOP/s (valid pairs) on 1 B200",
+            "metric": METRIC,
             "value": round(v, 6), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(el * 1e3, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
