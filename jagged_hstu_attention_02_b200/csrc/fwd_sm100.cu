@@ -114,8 +114,9 @@ __device__ __forceinline__ void report_timeout(const DevParams &p)
 // LayerNorm gradient is sensitive to the error of Y).  Without SPLIT, A has two TMEM
 // buffers of 64 columns; with SPLIT one buffer of 128 (per 32-key quarter w: hi at
 // 32w..32w+15, lo at 32w+16..32w+31).
-// One 32-row x 32-key block of the epilogue (thread = row = TMEM lane): the bias, SiLU, the
-// mask, and A into TMEM.  The mode choices are template parameters, so the body has no
+// Training: one 32-row x 32-key block of the epilogue (thread = row = TMEM lane): the bias,
+// SiLU, the mask, and A (hi and lo parts) into TMEM, in fp32 with the accurate sigmoid.
+// The inference body is fwd_quarter_inf.  The mode choices are template parameters, so the body has no
 // branch and the compiler can overlap the loads and arithmetic of neighbouring keys:
 //   TM   time bias: 0 one bucket, 1 one boundary, 2 lookup table, 3 64-bit search
 //   RD   rel index rbase - c without clamping
@@ -140,7 +141,7 @@ struct FwdEpi {
     int64_t tsi;               // the row's stamp
 };
 
-template <int TM, bool RD, bool FULL, bool SPLIT>
+template <int TM, bool RD, bool FULL>
 __device__ __forceinline__ void fwd_quarter(const FwdEpi &e, const HalfTime &ht, uint32_t vmask)
 {
     // one-boundary test as a single unsigned compare: the key is in the lower bucket when
@@ -184,43 +185,26 @@ __device__ __forceinline__ void fwd_quarter(const FwdEpi &e, const HalfTime &ht,
         tmem_wait_ld();
         reg_fence(ra);
         const uint32_t vb = vmask >> cb;
-        uint32_t pk[2];
-        if constexpr (SPLIT) {
-            uint32_t plo[2];
+        uint32_t pk[2], plo[2];
 #pragma unroll
-            for (int c2 = 0; c2 < 2; ++c2) {
-                const float2 h = __ffma2_rn(ha2, make_float2(__uint_as_float(ra[2 * c2]),
-                                                             __uint_as_float(ra[2 * c2 + 1])),
-                                            bh[c2]);
-                float a[2];
+        for (int c2 = 0; c2 < 2; ++c2) {
+            const float2 h = __ffma2_rn(ha2, make_float2(__uint_as_float(ra[2 * c2]),
+                                                         __uint_as_float(ra[2 * c2 + 1])),
+                                        bh[c2]);
+            float a[2];
 #pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    const int c = 2 * c2 + q;
-                    const float xs = 2.0f * (q ? h.y : h.x);
-                    const float v = xs * __fdividef(1.0f, 1.0f + __expf(-xs));
-                    a[q] = (FULL || ((vb >> c) & 1u)) ? v : 0.f;
-                }
-                pk[c2] = pack_bf16x2(a[0], a[1]);
-                plo[c2] = pack_bf16x2(a[0] - __uint_as_float(pk[c2] << 16),
-                                      a[1] - __uint_as_float(pk[c2] & 0xFFFF0000u));
+            for (int q = 0; q < 2; ++q) {
+                const int c = 2 * c2 + q;
+                const float xs = 2.0f * (q ? h.y : h.x);
+                const float v = xs * __fdividef(1.0f, 1.0f + __expf(-xs));
+                a[q] = (FULL || ((vb >> c) & 1u)) ? v : 0.f;
             }
-            tmem_st2(e.t_a + ch * 2, pk);
-            tmem_st2(e.t_a + 16 + ch * 2, plo);
-        } else {
-#pragma unroll
-            for (int c2 = 0; c2 < 2; ++c2) {
-                const float2 x = __ffma2_rn(ha2, make_float2(__uint_as_float(ra[2 * c2]),
-                                                             __uint_as_float(ra[2 * c2 + 1])),
-                                            bh[c2]);
-                const uint32_t h2 = __byte_perm(__float_as_uint(x.x), __float_as_uint(x.y), 0x7632);
-                uint32_t a2 = fma_bf16x2(h2, tanh_bf16x2(h2), h2);
-                if (!FULL)
-                    a2 &= (((vb >> (2 * c2)) & 1u) ? 0x0000FFFFu : 0u) |
-                          (((vb >> (2 * c2 + 1)) & 1u) ? 0xFFFF0000u : 0u);
-                pk[c2] = a2;
-            }
-            tmem_st2(e.t_a + ch * 2, pk);
+            pk[c2] = pack_bf16x2(a[0], a[1]);
+            plo[c2] = pack_bf16x2(a[0] - __uint_as_float(pk[c2] << 16),
+                                  a[1] - __uint_as_float(pk[c2] & 0xFFFF0000u));
         }
+        tmem_st2(e.t_a + ch * 2, pk);
+        tmem_st2(e.t_a + 16 + ch * 2, plo);
     }
 }
 
@@ -719,7 +703,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     // this quarter's A columns (SPLIT: hi and lo parts, 32 columns)
                     tmem_zero16(e.t_a);
                     if constexpr (SPLIT) tmem_zero16(e.t_a + 16);
-                } else if (!SPLIT) {
+                } else if constexpr (!SPLIT) {
                     if (tmode == 3) fwd_quarter_inf<3, false, false>(e, ht, vmask);
                     else if (!rdirect) {
                         if (tmode == 0) fwd_quarter_inf<0, false, false>(e, ht, vmask);
@@ -733,19 +717,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         else fwd_quarter_inf<2, true, false>(e, ht, vmask);
                     }
                 } else if (tmode == 3) {
-                    fwd_quarter<3, false, false, SPLIT>(e, ht, vmask);
+                    fwd_quarter<3, false, false>(e, ht, vmask);
                 } else if (full && rdirect) {
-                    if (tmode == 0) fwd_quarter<0, true, true, SPLIT>(e, ht, vmask);
-                    else if (tmode == 1) fwd_quarter<1, true, true, SPLIT>(e, ht, vmask);
-                    else fwd_quarter<2, true, true, SPLIT>(e, ht, vmask);
+                    if (tmode == 0) fwd_quarter<0, true, true>(e, ht, vmask);
+                    else if (tmode == 1) fwd_quarter<1, true, true>(e, ht, vmask);
+                    else fwd_quarter<2, true, true>(e, ht, vmask);
                 } else if (rdirect) {
-                    if (tmode == 0) fwd_quarter<0, true, false, SPLIT>(e, ht, vmask);
-                    else if (tmode == 1) fwd_quarter<1, true, false, SPLIT>(e, ht, vmask);
-                    else fwd_quarter<2, true, false, SPLIT>(e, ht, vmask);
+                    if (tmode == 0) fwd_quarter<0, true, false>(e, ht, vmask);
+                    else if (tmode == 1) fwd_quarter<1, true, false>(e, ht, vmask);
+                    else fwd_quarter<2, true, false>(e, ht, vmask);
                 } else {
-                    if (tmode == 0) fwd_quarter<0, false, false, SPLIT>(e, ht, vmask);
-                    else if (tmode == 1) fwd_quarter<1, false, false, SPLIT>(e, ht, vmask);
-                    else fwd_quarter<2, false, false, SPLIT>(e, ht, vmask);
+                    if (tmode == 0) fwd_quarter<0, false, false>(e, ht, vmask);
+                    else if (tmode == 1) fwd_quarter<1, false, false>(e, ht, vmask);
+                    else fwd_quarter<2, false, false>(e, ht, vmask);
                 }
                 tc_fence_before();
                 warp_arrive(&bars[S_FREE + st]);      // S has been read
