@@ -54,6 +54,8 @@ SMALL_CASES = [
     # head dims the tensor-core forward runs zero-padded to 64 / 128
     ("bf16-d96-d48", [33, 260, 129], 2, 96, 48, "bf16", [1, 4, 0], [2, 9, 1], 0, 261, 128),
     ("bf16-d16-d112", [150, 7, 300], 3, 16, 112, "bf16", 2, [3, 0, 30], 60, 61, 128),
+    # the widest rows (H * d_v = 2048) and the largest time table (256 buckets)
+    ("bf16-max-width", [70, 300], 16, 128, 128, "bf16", [2, 0], [5, 17], 0, 301, 256),
 ]
 
 
