@@ -3,12 +3,13 @@
 // A work unit is (128-row query tile, sequence, head).  For every key tile of 128 that holds
 // a valid pair:  S = Q K^T on tcgen05 (bf16 operands staged by TMA in 128-byte-swizzled
 // shared memory, fp32 accumulator in TMEM); the epilogue warps read S from TMEM and form
-// A = mask ? SiLU(alpha*S + b) : 0 in fp32, where b is the relative-position plus bucketed
-// time bias and the mask is applied after the nonlinearity, never as -inf before it ("HSTU
+// A = mask ? SiLU(alpha*S + b) : 0, where b is the relative-position plus bucketed time
+// bias and the mask is applied after the nonlinearity, never as -inf before it ("HSTU
 // tensor by tensor: SiLU aggregation, temporal bias and gating", sections "Similar shape,
-// different aggregation" and "Do not copy softmax masking mechanically"); A is rounded to
-// bf16 and written into its own TMEM columns (two elements per 32-bit column), and tcgen05
-// adds A V into an fp32 output accumulator in TMEM with A read from TMEM.  The 1/N scale
+// different aggregation" and "Do not copy softmax masking mechanically") -- in packed bf16
+// pairs for inference, in fp32 with A split into bf16 hi + lo parts for training; A goes
+// into its own TMEM columns (two bf16 elements per 32-bit column), and tcgen05 adds A V
+// into an fp32 output accumulator in TMEM with A read from TMEM.  The 1/N scale
 // ("HSTU-MUSA: HSTU for Moore Threads (MUSA)", "Accuracy Alignment": N = batch max_seqlen)
 // is applied once to the accumulator; Y goes to global memory in fp32.
 //
@@ -27,9 +28,11 @@
 // Bias evaluation per (row, 32-key quarter tile):  the time bucket is computed once for
 // the smallest and largest |dt| the quarter can produce (from its timestamp range); when
 // both agree (the common case away from the diagonal) the time bias is a per-row constant.
-// The rel index runs p(i)-j down a contiguous window of the table when no clamping occurs.
-// Mask evaluation is skipped on tiles the mask covers fully.  Every wait is bounded; a
-// timeout sets HSTU_DEV_WAIT_TIMEOUT and the CTA unwinds.
+// The rel index runs p(i)-j down a contiguous window of the table when no clamping occurs
+// (inference: a guard-banded table of bf16 key pairs, one load per two keys).  Blocks
+// without a valid pair only write zeros; the training body skips the mask on fully valid
+// blocks, the inference body always applies it (one byte permute per key pair).  Every
+// wait is bounded; a timeout sets HSTU_DEV_WAIT_TIMEOUT and the CTA unwinds.
 #include <cudaTypedefs.h>
 
 #include <atomic>
