@@ -8,7 +8,8 @@
 //   - the LayerNorm of the input tokens (no affine) that precedes the projection.
 //
 // GEMM: C[M, N] = A[M, K] B[K, N], bf16 operands (A row-major: K-major; B row-major: N-major),
-// fp32 accumulation in TMEM.  Persistent CTAs take 128 x BN output tiles in a static order;
+// fp32 accumulation in TMEM.  Persistent CTAs take 128 x BN output tiles (BN = 128) in a
+// static order;
 // warp 0 lane 0 streams 64-wide K slices of A and B through a four-stage ring with TMA
 // (128-byte swizzle), warp 1 lane 0 issues tcgen05.mma into one of two TMEM accumulators,
 // warps 2-9 read the other accumulator back (two warps per TMEM lane quarter, each half of
@@ -371,7 +372,9 @@ cudaError_t launch_gemm(const void *A, const void *B, int M, int N, int K, const
     if (M <= 0) return cudaSuccess;
     GemmArgs a;
     std::memset(&a, 0, sizeof(a));
-    const int BN = N >= 256 ? 256 : 128;
+    // 128-wide tiles: twice the tiles of 256-wide ones, so the last wave of the persistent
+    // grid is fuller (the U/V/Q/K projection of 10.9k tokens: 0.0256 against 0.0267 ms)
+    constexpr int BN = 128;
     if (!encode_2d(&a.ta, A, M, K, GBM) || !encode_2d(&a.tb, B, K, N, GBK))
         return cudaErrorInvalidValue;
     a.M = M;
@@ -385,7 +388,7 @@ cudaError_t launch_gemm(const void *A, const void *B, int M, int N, int K, const
     for (int s = 0; s < nseg; ++s) a.out[s] = reinterpret_cast<__nv_bfloat16 *>(outs[s]);
     a.status = status;
     a.wait_limit = wait_limit;
-    return BN == 256 ? run_gemm<256>(a, st) : run_gemm<128>(a, st);
+    return run_gemm<BN>(a, st);
 }
 
 }  // namespace hstu
