@@ -10,11 +10,10 @@
 // GEMM: C[M, N] = A[M, K] B[K, N], bf16 operands (A row-major: K-major; B row-major: N-major),
 // fp32 accumulation in TMEM.  Persistent CTAs take 128 x BN output tiles (BN = 128) in a
 // static order; warp 0 lane 0 streams 64-wide K slices of A and B through a four-stage ring
-// with TMA
-// (128-byte swizzle), warp 1 lane 0 issues tcgen05.mma into one of two TMEM accumulators,
-// warps 2-9 read the other accumulator back (two warps per TMEM lane quarter, each half of
-// the columns; thread = row = TMEM lane) and write bf16 outputs, so a tile's epilogue
-// overlaps the next tile's MMAs.  Every wait is bounded.
+// with TMA (128-byte swizzle), warp 1 lane 0 issues tcgen05.mma into one of two TMEM
+// accumulators, warps 2-9 read the other accumulator back (two warps per TMEM lane quarter,
+// each half of the columns; thread = row = TMEM lane) and write bf16 outputs, so a tile's
+// epilogue overlaps the next tile's MMAs.  Every wait is bounded.
 #include <cudaTypedefs.h>
 
 #include <cstring>
